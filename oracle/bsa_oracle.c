@@ -1,0 +1,250 @@
+/*
+ * BSA forward oracle: a plain, slow, fp64 CPU statement of mesh-aligned
+ * block-sparse attention, written step by step from the MOSAIC note
+ * ("(Sparse) Attention to the Details", papernotes.org ICML 2026 page,
+ * section "Mesh-aligned Block-Sparse Attention (BSA)"):
+ *
+ *   partition the N NESTED tokens into m contiguous blocks, pool each block
+ *   (phi = mean), (a) compressed branch softmax(q̄_i·k̄_j/sqrt(d)) block to
+ *   block, broadcast to the tokens of block i, (b) selection branch: each
+ *   query block keeps the top-n key blocks by compressed score and runs
+ *   full-resolution attention over their tokens, (c) local branch: standard
+ *   attention over a sliding window, and o = g_CG o_CG + g_FG o_FG + g_L o_L.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or
+ * load this file or its library; only the tests, the package's smoke check
+ * and the benchmark's CPU-baseline leg use it. It shares no code with the
+ * CUDA library.
+ *
+ * Readings where the note is silent (each also listed in the design notes):
+ *  - phi is the arithmetic mean over the block's tokens.
+ *  - o_CG of query block i is sum_j softmax_j(z_ij) * v̄_j (pooled values),
+ *    identical for every token of block i.
+ *  - one scale s = 1/sqrt(d) (or the caller's) in all three branches.
+ *  - top-n ranks the logits z_ij (softmax is monotone); equal logits go to
+ *    the lower block index; output order is (z descending, j ascending).
+ *  - no causal mask; selected blocks may overlap the local window, the two
+ *    branches keep separate softmaxes.
+ *  - the local window is block aligned, blocks max(0,i-w) .. min(m-1,i+w),
+ *    clamped at the ends of the NESTED sequence (no wrap-around).
+ *  - gates are given per token, order (CG, FG, L), not normalised.
+ *
+ * All arrays are row-major and describe ONE (batch, head) slab:
+ *   q, k, v [N][d], gates [N][3], pooled [m][d], idx [m][n] (int32).
+ * Functions return 0 on success, -1 on bad arguments.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---- step 1-2: block partition and pooling phi (mean) ------------------ */
+
+/* xbar[j][c] = (1/B) * sum over the B tokens of block j of x[t][c];
+ * block j holds tokens j*B .. j*B+B-1 (one parent pixel in NESTED order). */
+int oracle_pool(int64_t n_tokens, int64_t d, int64_t block,
+                const double *x, double *xbar)
+{
+    if (n_tokens <= 0 || d <= 0 || block <= 0 || n_tokens % block != 0) return -1;
+    int64_t m = n_tokens / block;
+    for (int64_t j = 0; j < m; ++j) {
+        for (int64_t c = 0; c < d; ++c) {
+            double s = 0.0;
+            for (int64_t t = j * block; t < (j + 1) * block; ++t) s += x[t * d + c];
+            xbar[j * d + c] = s / (double)block;
+        }
+    }
+    return 0;
+}
+
+/* ---- step 3-4: compressed branch and top-n selection ------------------- */
+
+typedef struct { double z; int32_t j; } scored_block;
+
+/* Sort key (-z, j): larger logit first, equal logits by lower block index. */
+static int by_score_then_index(const void *pa, const void *pb)
+{
+    const scored_block *a = (const scored_block *)pa, *b = (const scored_block *)pb;
+    if (a->z > b->z) return -1;
+    if (a->z < b->z) return 1;
+    return (a->j < b->j) ? -1 : (a->j > b->j);
+}
+
+/*
+ * For query blocks i in [r0, r1):
+ *   z_ij    = s * sum_c q̄_ic k̄_jc                     (j = 0 .. m-1)
+ *   ā_ij    = exp(z_ij - max_j z_ij) / sum_j exp(...)
+ *   o_cg_i  = sum_j ā_ij v̄_j
+ *   idx_i   = the n blocks first in the order (z desc, j asc)
+ *   gap_i   = z_(n) - z_(n+1) in that order, +inf when n == m
+ * Output rows are relative to r0. z_out (nullable) receives the logits.
+ */
+int oracle_compressed_rows(int64_t m, int64_t d, int64_t n, double scale,
+                           const double *qbar, const double *kbar, const double *vbar,
+                           int64_t r0, int64_t r1,
+                           double *o_cg, int32_t *idx, double *gap, double *z_out)
+{
+    if (m <= 0 || d <= 0 || n < 1 || n > m || r0 < 0 || r1 > m || r0 > r1) return -1;
+    int64_t rows = r1 - r0;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t i = r0 + r;
+        scored_block *sb = (scored_block *)malloc((size_t)m * sizeof(scored_block));
+        double *w = (double *)malloc((size_t)m * sizeof(double));
+        if (!sb || !w) { free(sb); free(w); bad = 1; continue; }
+        double zmax = -INFINITY;
+        for (int64_t j = 0; j < m; ++j) {
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += qbar[i * d + c] * kbar[j * d + c];
+            double z = scale * dot;
+            sb[j].z = z;
+            sb[j].j = (int32_t)j;
+            if (z_out) z_out[r * m + j] = z;
+            if (z > zmax) zmax = z;
+        }
+        double denom = 0.0;
+        for (int64_t j = 0; j < m; ++j) { w[j] = exp(sb[j].z - zmax); denom += w[j]; }
+        for (int64_t c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < m; ++j) acc += w[j] * vbar[j * d + c];
+            o_cg[r * d + c] = acc / denom;
+        }
+        qsort(sb, (size_t)m, sizeof(scored_block), by_score_then_index);
+        for (int64_t t = 0; t < n; ++t) idx[r * n + t] = sb[t].j;
+        gap[r] = (n < m) ? sb[n - 1].z - sb[n].z : INFINITY;
+        free(sb);
+        free(w);
+    }
+    return bad ? -1 : 0;
+}
+
+/* ---- step 5-7: selection branch, local branch, gated combine ----------- */
+
+/* Softmax attention of one query row over the tokens of the listed blocks:
+ * out[c] = sum_u p_u v_uc, p_u = softmax_u(s * q·k_u). */
+static void attend_blocks(int64_t d, int64_t block, double scale, const double *qt,
+                          const double *k, const double *v,
+                          const int64_t *blocks, int64_t nb, double *scores, double *out)
+{
+    int64_t nk = nb * block;
+    double smax = -INFINITY;
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int64_t t = 0; t < block; ++t) {
+            int64_t u = blocks[b] * block + t;
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += qt[c] * k[u * d + c];
+            double s = scale * dot;
+            scores[b * block + t] = s;
+            if (s > smax) smax = s;
+        }
+    }
+    double denom = 0.0;
+    for (int64_t e = 0; e < nk; ++e) { scores[e] = exp(scores[e] - smax); denom += scores[e]; }
+    for (int64_t c = 0; c < d; ++c) out[c] = 0.0;
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int64_t t = 0; t < block; ++t) {
+            int64_t u = blocks[b] * block + t;
+            double p = scores[b * block + t] / denom;
+            for (int64_t c = 0; c < d; ++c) out[c] += p * v[u * d + c];
+        }
+    }
+}
+
+/*
+ * For query blocks i in [qb0, qb1) and every token t of block i:
+ *   o_fg_t = attention over the tokens of blocks idx[i][0..n-1]
+ *   o_l_t  = attention over the tokens of blocks max(0,i-w) .. min(m-1,i+w)
+ *   out_t  = g_t0 * o_cg[i] + g_t1 * o_fg_t + g_t2 * o_l_t
+ * o_cg is the block-level compressed output [m][d]; idx is [m][n] with
+ * entries in [0, m). Output rows are relative to token qb0*block.
+ * o_fg_out / o_l_out are nullable.
+ */
+int oracle_fine_rows(int64_t n_tokens, int64_t d, int64_t block, int64_t n, int64_t w,
+                     double scale, const double *q, const double *k, const double *v,
+                     const double *gates, const double *o_cg, const int32_t *idx,
+                     int64_t qb0, int64_t qb1,
+                     double *out, double *o_fg_out, double *o_l_out)
+{
+    if (n_tokens <= 0 || d <= 0 || block <= 0 || n_tokens % block != 0) return -1;
+    int64_t m = n_tokens / block;
+    if (n < 1 || n > m || w < 0 || qb0 < 0 || qb1 > m || qb0 > qb1) return -1;
+    for (int64_t i = qb0; i < qb1; ++i)
+        for (int64_t t = 0; t < n; ++t)
+            if (idx[i * n + t] < 0 || idx[i * n + t] >= m) return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = qb0; i < qb1; ++i) {
+        int64_t lo = (i - w < 0) ? 0 : i - w;
+        int64_t hi = (i + w > m - 1) ? m - 1 : i + w;
+        int64_t nl = hi - lo + 1;
+        int64_t nmax = (n > nl) ? n : nl;
+        int64_t *sel = (int64_t *)malloc((size_t)n * sizeof(int64_t));
+        int64_t *loc = (int64_t *)malloc((size_t)nl * sizeof(int64_t));
+        double *scores = (double *)malloc((size_t)(nmax * block) * sizeof(double));
+        double *ofg = (double *)malloc((size_t)d * sizeof(double));
+        double *ol = (double *)malloc((size_t)d * sizeof(double));
+        if (!sel || !loc || !scores || !ofg || !ol) {
+            free(sel); free(loc); free(scores); free(ofg); free(ol); bad = 1; continue;
+        }
+        for (int64_t t = 0; t < n; ++t) sel[t] = idx[i * n + t];
+        for (int64_t b = 0; b < nl; ++b) loc[b] = lo + b;
+        for (int64_t t = i * block; t < (i + 1) * block; ++t) {
+            const double *qt = q + t * d;
+            attend_blocks(d, block, scale, qt, k, v, sel, n, scores, ofg);
+            attend_blocks(d, block, scale, qt, k, v, loc, nl, scores, ol);
+            int64_t r = t - qb0 * block;
+            const double *g = gates + t * 3;
+            for (int64_t c = 0; c < d; ++c) {
+                out[r * d + c] = g[0] * o_cg[i * d + c] + g[1] * ofg[c] + g[2] * ol[c];
+                if (o_fg_out) o_fg_out[r * d + c] = ofg[c];
+                if (o_l_out) o_l_out[r * d + c] = ol[c];
+            }
+        }
+        free(sel); free(loc); free(scores); free(ofg); free(ol);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * The whole forward pass of one slab, steps 1-7 in order. When forced_idx is
+ * non-null the selection branch uses it instead of the computed top-n (the
+ * computed indices and gaps are still returned), so that a caller can
+ * re-evaluate outputs on another implementation's near-tie choices.
+ * Outputs: out [N][d]; nullable extras: qbar/kbar/vbar [m][d], o_cg [m][d],
+ * idx [m][n], gap [m].
+ */
+int oracle_forward_slab(int64_t n_tokens, int64_t d, int64_t block, int64_t n, int64_t w,
+                        double scale, const double *q, const double *k, const double *v,
+                        const double *gates, const int32_t *forced_idx,
+                        double *out, double *qbar_out, double *kbar_out, double *vbar_out,
+                        double *o_cg_out, int32_t *idx_out, double *gap_out)
+{
+    if (n_tokens <= 0 || d <= 0 || block <= 0 || n_tokens % block != 0) return -1;
+    int64_t m = n_tokens / block;
+    if (n < 1 || n > m) return -1;
+    double *qb = (double *)malloc((size_t)(m * d) * sizeof(double));
+    double *kb = (double *)malloc((size_t)(m * d) * sizeof(double));
+    double *vb = (double *)malloc((size_t)(m * d) * sizeof(double));
+    double *ocg = (double *)malloc((size_t)(m * d) * sizeof(double));
+    int32_t *ix = (int32_t *)malloc((size_t)(m * n) * sizeof(int32_t));
+    double *gp = (double *)malloc((size_t)m * sizeof(double));
+    int rc = -1;
+    if (qb && kb && vb && ocg && ix && gp &&
+        oracle_pool(n_tokens, d, block, q, qb) == 0 &&
+        oracle_pool(n_tokens, d, block, k, kb) == 0 &&
+        oracle_pool(n_tokens, d, block, v, vb) == 0 &&
+        oracle_compressed_rows(m, d, n, scale, qb, kb, vb, 0, m, ocg, ix, gp, NULL) == 0 &&
+        oracle_fine_rows(n_tokens, d, block, n, w, scale, q, k, v, gates, ocg,
+                         forced_idx ? forced_idx : ix, 0, m, out, NULL, NULL) == 0) {
+        rc = 0;
+        if (qbar_out) memcpy(qbar_out, qb, (size_t)(m * d) * sizeof(double));
+        if (kbar_out) memcpy(kbar_out, kb, (size_t)(m * d) * sizeof(double));
+        if (vbar_out) memcpy(vbar_out, vb, (size_t)(m * d) * sizeof(double));
+        if (o_cg_out) memcpy(o_cg_out, ocg, (size_t)(m * d) * sizeof(double));
+        if (idx_out) memcpy(idx_out, ix, (size_t)(m * n) * sizeof(int32_t));
+        if (gap_out) memcpy(gap_out, gp, (size_t)m * sizeof(double));
+    }
+    free(qb); free(kb); free(vb); free(ocg); free(ix); free(gp);
+    return rc;
+}

@@ -1,0 +1,59 @@
+"""Plant plausible mistakes in a copy of the oracle (CPU only) and check that
+the pin suite notices every one of them. The oracle source itself is never
+modified: each mutant is compiled from a temporary copy."""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins as pins
+from oracle import build as obuild
+
+SRC = open(obuild.SRC).read()
+
+MUTANTS = {
+    "z_transposed": ("qbar[i * d + c] * kbar[j * d + c]", "qbar[j * d + c] * kbar[i * d + c]"),
+    "z_scale_dropped": ("double z = scale * dot;", "double z = dot;"),
+    "compressed_wrong_values": ("acc += w[j] * vbar[j * d + c]", "acc += w[j] * kbar[j * d + c]"),
+    "compressed_not_normalised": ("o_cg[r * d + c] = acc / denom;", "o_cg[r * d + c] = acc;"),
+    "ties_to_higher_index": ("return (a->j < b->j) ? -1 : (a->j > b->j);",
+                             "return (a->j > b->j) ? -1 : (a->j < b->j);"),
+    "topn_ascending": ("if (a->z > b->z) return -1;\n    if (a->z < b->z) return 1;",
+                       "if (a->z < b->z) return -1;\n    if (a->z > b->z) return 1;"),
+    "gap_wrong_ranks": ("sb[n - 1].z - sb[n].z", "sb[0].z - sb[n].z"),
+    "pool_divides_by_d": ("xbar[j * d + c] = s / (double)block;", "xbar[j * d + c] = s / (double)d;"),
+    "pool_skips_last_token": ("t < (j + 1) * block; ++t) s += x", "t < (j + 1) * block - 1; ++t) s += x"),
+    "window_right_edge_dropped": ("int64_t hi = (i + w > m - 1) ? m - 1 : i + w;",
+                                  "int64_t hi = (i + w > m - 1) ? m - 1 : i;"),
+    "window_wraps_left": ("int64_t lo = (i - w < 0) ? 0 : i - w;", "int64_t lo = (i - w < 0) ? i : i - w;"),
+    "fine_not_normalised": ("double p = scores[b * block + t] / denom;", "double p = scores[b * block + t];"),
+    "fine_no_scale": ("double s = scale * dot;", "double s = dot;"),
+    "selection_uses_row0": ("sel[t] = idx[i * n + t];", "sel[t] = idx[t];"),
+    "gates_fg_l_swapped": ("g[1] * ofg[c] + g[2] * ol[c]", "g[2] * ofg[c] + g[1] * ol[c]"),
+    "cg_term_dropped": ("g[0] * o_cg[i * d + c] + g[1]", "0.0 * o_cg[i * d + c] + g[1]"),
+    "cg_wrong_block": ("g[0] * o_cg[i * d + c]", "g[0] * o_cg[(m - 1 - i) * d + c]"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(tmp_path, name):
+    old, new = MUTANTS[name]
+    assert SRC.count(old) == 1, f"mutation anchor for {name} not unique in the oracle source"
+    src = tmp_path / "mutant.c"
+    src.write_text(SRC.replace(old, new))
+    lib = oracle.load(obuild.build(str(src), str(tmp_path / "libmutant.so"), force=True))
+    caught = []
+    for check in pins.ALL_CHECKS:
+        try:
+            check(lib)
+        except (AssertionError, ValueError) as e:
+            caught.append(f"{check.__name__}: {str(e)[:80]}")
+    assert caught, f"no pin detects mutant {name}"
+
+
+def test_unmutated_copy_passes(tmp_path):
+    src = tmp_path / "copy.c"
+    src.write_text(SRC)
+    lib = oracle.load(obuild.build(str(src), str(tmp_path / "libcopy.so"), force=True))
+    for check in pins.ALL_CHECKS:
+        check(lib)
