@@ -1,0 +1,415 @@
+"""Benchmark of the BSA forward pass (pool -> compress/select -> fine attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload nside128] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of the workload's
+synthetic inputs, resident in HBM. Prints ONE JSON line on rank 0.
+
+Multi-GPU (torchrun, one rank per GPU): the (batch, head) slabs of BSA are
+independent problems, so every rank runs its own full batch with no
+collective on the data path ("scaling": "weak"); the step time is the max
+over ranks of the device-timed region and `value` counts all ranks' tokens.
+
+--impl reference times the fp64 CPU oracle on the host cores (rank 0 only),
+each step a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_spherical_b200.configs import CONFIGS, HEADLINE  # noqa: E402
+
+METRIC = "BSA fwd tokens/s & TFLOP/s at Nside=128 (1 B200); % of BF16 tensor/HBM peak"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SM_COUNT_B200 = 148
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(cfg):
+    return {"workload": cfg.name, "nside": cfg.nside, "n_tokens": cfg.n_tokens, "batch": cfg.batch,
+            "heads": cfg.heads, "head_dim": cfg.head_dim, "block_size": cfg.block_size,
+            "n_blocks": cfg.n_blocks, "top_n": cfg.top_n, "window_blocks": cfg.window_blocks,
+            "seed": cfg.seed,
+            "l2": f"inputs larger than L2: q, k, v {cfg.slabs * cfg.n_tokens * cfg.head_dim * cfg.elt_bytes / 1e6:.0f} MB each"}
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of SM clock and throttle reasons during the timed region."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "utilization.gpu",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        cmd = ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        if self.gpu_id:
+            cmd += ["--id=" + self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        rows = []
+        for l in self.lines:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        loaded = [r for r in rows if r[2] >= 50.0] or rows
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in loaded:
+            for n, v in zip(names, r[3]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(loaded)}
+
+
+# ----------------------------------------------------------------- oracle leg
+
+_SLAB_CACHE = {}
+
+
+def oracle_sample(cfg, target_s: float, slab: int = 0, lib=None):
+    """Time the oracle on a bounded sample of one slab; return (tokens/s, description, seconds)."""
+    import oracle
+    from block_sparse_spherical_b200.synthetic import make_slab
+    lib = lib or oracle.load()
+    key = (cfg.name, slab)
+    if key not in _SLAB_CACHE:
+        s = make_slab(cfg, slab)
+        _SLAB_CACHE[key] = tuple(x.astype(np.float64) for x in (s.q, s.k, s.v, s.gates))
+    q, k, v, g = _SLAB_CACHE[key]
+    bk, n, w, m = cfg.block_size, cfg.top_n, cfg.window_blocks, cfg.n_blocks
+    t0 = time.perf_counter()
+    qb, kb, vb = (oracle.pool(x, bk, lib=lib) for x in (q, k, v))
+    t_pool = time.perf_counter() - t0
+
+    def run(nblk):
+        t = time.perf_counter()
+        c = oracle.compressed_rows(qb, kb, vb, n, rows=(0, nblk), lib=lib)
+        ocg = np.zeros((m, cfg.head_dim))
+        ocg[:nblk] = c["o_cg"]
+        idx = np.zeros((m, n), np.int32)
+        idx[:nblk] = c["idx"]
+        oracle.fine_rows(q, k, v, g, ocg, idx, bk, n, w, qblocks=(0, nblk), lib=lib)
+        return time.perf_counter() - t
+
+    probe = min(m, 8)
+    t_probe = run(probe)
+    nblk = int(min(m, max(probe, probe * target_s / max(t_probe, 1e-6))))
+    t_run = run(nblk) if nblk > probe else t_probe
+    elapsed = t_run + t_pool * nblk / m
+    tokens = nblk * bk
+    desc = (f"slab {slab} of {cfg.name}: query blocks 0..{nblk - 1} ({tokens} tokens; compressed rows "
+            f"over all {m} key blocks, selection+local+combine), pooling of the slab pro-rated by {nblk}/{m}")
+    return tokens / elapsed, desc, elapsed
+
+
+def omp_threads():
+    return int(os.environ.get("OMP_NUM_THREADS") or os.cpu_count() or 1)
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return
+    os.environ.setdefault("OMP_NUM_THREADS", str(os.cpu_count() or 1))
+    import oracle
+    lib = oracle.load()
+    per_step = float(os.environ.get("BSA_ORACLE_STEP_S", "3.0"))
+    for _ in range(args.warmup):
+        oracle_sample(cfg, min(per_step, 0.5), lib=lib)
+    rates, descs, secs = [], [], 0.0
+    for _ in range(args.steps):
+        r, d, e = oracle_sample(cfg, per_step, lib=lib)
+        rates.append(r)
+        descs.append(d)
+        secs += e
+    value = statistics.median(rates)
+    tokens_step = cfg.slabs * cfg.n_tokens
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tokens_step / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(cfg),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
+                             "sample": descs[-1] + "; value = median over steps, ms_per_step extrapolated "
+                                                   "to the whole workload"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def traffic_for(kernel_file: str, key: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f).get(key)
+    if not d:
+        return None
+    src = os.path.join(ROOT, "block_sparse_spherical_b200", "csrc", kernel_file)
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if d.get("source_sha") != sha:
+        return None
+    return d.get("bytes_per_launch_full_workload")
+
+
+def run_ours(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from block_sparse_spherical_b200 import abi, api
+    from block_sparse_spherical_b200.synthetic import make_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    # independent problem per rank: same workload, rank-offset seed
+    rcfg = cfg.with_(seed=cfg.seed + 1000 * rank) if rank else cfg
+    qh, kh, vh, gh = make_inputs(rcfg)
+    tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
+
+    def host(a):
+        t = torch.from_numpy(a)
+        return t.view(torch.bfloat16) if cfg.dtype == "bf16" else t
+
+    q, k, v, g = (host(a).to(dev) for a in (qh, kh, vh, gh))
+    stream = torch.cuda.current_stream(dev)
+    bsa = api.BSA.from_config(cfg, device=dev)
+    c = bsa.cfg
+    m, d, n = cfg.n_blocks, cfg.head_dim, cfg.top_n
+    qb, kb, vb, ocg = (torch.empty((cfg.batch, cfg.heads, m, d), dtype=torch.float32, device=dev) for _ in range(4))
+    idx = torch.empty((cfg.batch, cfg.heads, m, n), dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        abi.bsa_pool(c, q, k, v, qb, kb, vb, stream)
+        if evs:
+            evs[1].record(stream)
+        abi.bsa_compress_select(c, qb, kb, vb, ocg, idx, stream)
+        if evs:
+            evs[2].record(stream)
+        abi.bsa_fine_attention(c, q, k, v, g, ocg, idx, out, status, stream)
+        if evs:
+            evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if abi.bsa_check_status(status, stream) != 0:
+        raise RuntimeError("kernel status word reports an error")
+
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid) if rank == 0 else None
+    except Exception:
+        gpu_id = None
+    sampler = ClockSampler(gpu_id) if rank == 0 else None
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.5)
+    for s in range(args.steps):
+        step(evs[s])
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    if world > 1:
+        dist.barrier()
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    k_ms = {"pool": [e[0].elapsed_time(e[1]) for e in evs],
+            "compress_select": [e[1].elapsed_time(e[2]) for e in evs],
+            "fine_attention": [e[2].elapsed_time(e[3]) for e in evs]}
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    if abi.bsa_check_status(status, stream) != 0:
+        raise RuntimeError("kernel status word reports an error")
+
+    # ---- end to end through the public API with host buffers (pinned), rank-local
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp, gp = (host(a).pin_memory() for a in (qh, kh, vh, gh))
+        outp = torch.empty(out.shape, dtype=tdt).pin_memory()
+        qd, kd, vd, gd = (torch.empty_like(x) for x in (q, k, v, g))
+
+        def e2e_step():
+            for dst, src in ((qd, qp), (kd, kp), (vd, vp), (gd, gp)):
+                dst.copy_(src, non_blocking=True)
+            o = bsa(qd, kd, vd, gd, out=out)
+            outp.copy_(o, non_blocking=True)
+
+        e2e_steps = max(3, args.steps // 4)
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        te = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp, gp))
+        e2e = {"value": world * e2e_steps * cfg.slabs * cfg.n_tokens / (float(te.item()) / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": outp.numel() * outp.element_size(),
+               "steps": e2e_steps, "api": "api.BSA.__call__ -> bsa_forward (C ABI)"}
+        if bsa.check_status() != 0:
+            raise RuntimeError("kernel status word reports an error")
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    tokens_step = cfg.slabs * cfg.n_tokens
+    ms_step = total_ms / args.steps
+    value = world * tokens_step / (ms_step / 1e3)
+    fine_flops, comp_flops = cfg.fine_flops(), cfg.compressed_flops()
+    mean = {kname: statistics.mean(v) for kname, v in k_ms.items()}
+    fine_tflops = fine_flops / (mean["fine_attention"] / 1e3) / 1e12
+    pool_gbs = cfg.pool_bytes() / (mean["pool"] / 1e3) / 1e9
+    comp_tflops = comp_flops / (mean["compress_select"] / 1e3) / 1e12
+    comp_gbs = cfg.compress_min_bytes() / (mean["compress_select"] / 1e3) / 1e9
+    fine_gbs = cfg.fused_min_bytes() / (mean["fine_attention"] / 1e3) / 1e9
+    sm_mhz = (clocks or {}).get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    fp32_peak = SM_COUNT_B200 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    tensor_peak = peaks["bf16_tflops_sustained"]
+    kernels = {
+        "pool": {"ms": mean["pool"], "bound": "hbm", "achieved_gbs": pool_gbs,
+                 "frac": pool_gbs / peaks["hbm_gbs"], "algorithmic_bytes": cfg.pool_bytes()},
+        "compress_select": {"ms": mean["compress_select"], "bound": "alu", "achieved_tflops_fp32": comp_tflops,
+                            "peak_tflops_fp32": fp32_peak, "frac": comp_tflops / fp32_peak,
+                            "achieved_gbs": comp_gbs, "frac_hbm": comp_gbs / peaks["hbm_gbs"],
+                            "algorithmic_flops": comp_flops},
+        "fine_attention": {"ms": mean["fine_attention"], "bound": "tensor", "achieved_tflops": fine_tflops,
+                           "frac": fine_tflops / tensor_peak, "achieved_gbs": fine_gbs,
+                           "algorithmic_flops": fine_flops},
+    }
+    dom = max(kernels, key=lambda kk: kernels[kk]["ms"])
+    kd = kernels[dom]
+    if kd["bound"] == "tensor":
+        roof = {"kernel": dom, "bound": "tensor", "achieved": kd["achieved_tflops"], "peak": tensor_peak,
+                "unit": "TFLOP/s", "frac": kd["frac"],
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long step loop)"}
+    elif kd["bound"] == "hbm":
+        roof = {"kernel": dom, "bound": "hbm", "achieved": kd["achieved_gbs"], "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": kd["frac"], "peak_source": f"{peak_src} hbm_gbs"}
+    else:
+        roof = {"kernel": dom, "bound": "alu", "achieved": kd["achieved_tflops_fp32"], "peak": fp32_peak,
+                "unit": "TFLOP/s", "frac": kd["frac"],
+                "peak_source": "148 SMs x 128 FP32 lanes x 2 flop x max SM clock"}
+    kfile = {"fine_attention": "attend_tc.cu", "pool": "pool.cu", "compress_select": "compress_select.cu"}[dom]
+    roof["traffic"] = traffic_for(kfile, f"{dom}:{cfg.name}")
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        os.environ.setdefault("OMP_NUM_THREADS", str(os.cpu_count() or 1))
+        rate, desc, secs = oracle_sample(cfg, float(os.environ.get("BSA_ORACLE_SAMPLE_S", "12")))
+        cpu = {"value": rate, "unit": UNIT, "cores": omp_threads(), "kind": "oracle",
+               "sample": desc, "seconds": secs}
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": dict(workload_config(cfg), parallelism=f"{world} independent replica(s), no collective"),
+            "tflops": world * (fine_flops + comp_flops) / (ms_step / 1e3) / 1e12,
+            "kernels": kernels, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 3 * args.steps, "clocks": clocks,
+            "gpu": torch.cuda.get_device_name(dev)}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = CONFIGS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+    else:
+        run_ours(args, cfg, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

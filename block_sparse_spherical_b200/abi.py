@@ -1,0 +1,130 @@
+"""Thin ctypes binding of libbsa.so (declared in include/bsa.h).
+
+Argument marshalling only: every function here passes device pointers,
+sizes and the current CUDA stream straight to the C ABI of the same name.
+All computation happens in the library's CUDA kernels; if the library is
+missing this module raises instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libbsa.so")
+
+BSA_OK = 0
+BSA_F32, BSA_BF16 = 0, 1
+STATUS_NAMES = {
+    0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "BSA_ERR_ALIGNMENT",
+    4: "BSA_ERR_CUDA", 5: "BSA_ERR_TIMEOUT", 6: "BSA_ERR_WORKSPACE", 7: "BSA_ERR_INDEX",
+}
+EXPORTS = ("bsa_pool", "bsa_compress_select", "bsa_fine_attention", "bsa_workspace_size",
+           "bsa_forward", "bsa_check_status", "bsa_status_string")
+
+
+class BsaConfig(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("n_tokens", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("block_size", ctypes.c_int32), ("top_n", ctypes.c_int32),
+                ("window_blocks", ctypes.c_int32), ("dtype", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class BsaError(RuntimeError):
+    def __init__(self, func: str, code: int):
+        self.code = code
+        super().__init__(f"{func} returned {STATUS_NAMES.get(code, code)}")
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libbsa.so once; raise loudly if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libbsa.so is not built ({LIB_PATH}); run python -m block_sparse_spherical_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, S, C = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(BsaConfig)
+    sig = {
+        "bsa_pool": [C, P, P, P, P, P, P, P],
+        "bsa_compress_select": [C, P, P, P, P, P, P],
+        "bsa_fine_attention": [C, P, P, P, P, P, P, P, P, P],
+        "bsa_workspace_size": [C, ctypes.POINTER(ctypes.c_size_t)],
+        "bsa_forward": [C, P, P, P, P, P, P, P, S, P],
+        "bsa_check_status": [P, P],
+        "bsa_status_string": [ctypes.c_int],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_char_p if name == "bsa_status_string" else ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def make_config(cfg, scale: float = 0.0) -> BsaConfig:
+    """BsaConfig from a configs.BSAConfig (or any object with the same fields)."""
+    return BsaConfig(cfg.batch, cfg.heads, cfg.n_tokens, cfg.head_dim, cfg.block_size, cfg.top_n,
+                     cfg.window_blocks, BSA_BF16 if cfg.dtype == "bf16" else BSA_F32, scale)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(name: str, rc: int) -> None:
+    if rc != BSA_OK:
+        raise BsaError(name, rc)
+
+
+def bsa_pool(cfg: BsaConfig, q, k, v, qbar, kbar, vbar, stream=None) -> None:
+    _check("bsa_pool", load().bsa_pool(ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(qbar),
+                                        _ptr(kbar), _ptr(vbar), _stream(stream)))
+
+
+def bsa_compress_select(cfg: BsaConfig, qbar, kbar, vbar, o_cg_block, sel_idx, stream=None) -> None:
+    _check("bsa_compress_select", load().bsa_compress_select(
+        ctypes.byref(cfg), _ptr(qbar), _ptr(kbar), _ptr(vbar), _ptr(o_cg_block), _ptr(sel_idx),
+        _stream(stream)))
+
+
+def bsa_fine_attention(cfg: BsaConfig, q, k, v, gates, o_cg_block, sel_idx, out, status_word=None,
+                       stream=None) -> None:
+    _check("bsa_fine_attention", load().bsa_fine_attention(
+        ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(o_cg_block), _ptr(sel_idx),
+        _ptr(out), _ptr(status_word), _stream(stream)))
+
+
+def bsa_workspace_size(cfg: BsaConfig) -> int:
+    n = ctypes.c_size_t(0)
+    _check("bsa_workspace_size", load().bsa_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def bsa_forward(cfg: BsaConfig, q, k, v, gates, out, sel_idx_out, workspace, workspace_bytes: int,
+                stream=None) -> None:
+    _check("bsa_forward", load().bsa_forward(
+        ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(out), _ptr(sel_idx_out),
+        _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def bsa_check_status(status_word, stream=None) -> int:
+    """Return the status code (0 = BSA_OK) after syncing `stream`; the word is reset."""
+    return load().bsa_check_status(_ptr(status_word), _stream(stream))
+
+
+def bsa_status_string(code: int) -> str:
+    return load().bsa_status_string(code).decode()

@@ -1,0 +1,127 @@
+"""torch-tensor front end of the BSA C ABI.
+
+PyTorch supplies device memory and the current stream; each call marshals
+tensors into one C-ABI call (abi.py) and the kernels in libbsa.so do all the
+work. Inputs must be contiguous CUDA tensors in the layouts of include/bsa.h.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import abi
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return abi.BSA_BF16
+    if t.dtype == torch.float32:
+        return abi.BSA_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _require(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def config_for(q: torch.Tensor, block_size: int, top_n: int, window_blocks: int = 1,
+               scale: float = 0.0) -> abi.BsaConfig:
+    b, h, n, d = q.shape
+    return abi.BsaConfig(b, h, n, d, block_size, top_n, window_blocks, _dtype_code(q), scale)
+
+
+class BSA:
+    """A BSA forward pass of fixed shape with its workspace held on the device.
+
+    Calling the object runs pool -> compress/select -> fine attention on the
+    current stream (three kernels) and returns `out` ([B, H, N, d], q's dtype).
+    """
+
+    def __init__(self, batch: int, heads: int, n_tokens: int, head_dim: int, block_size: int,
+                 top_n: int, window_blocks: int = 1, dtype=torch.bfloat16, scale: float = 0.0,
+                 device="cuda"):
+        self.cfg = abi.BsaConfig(batch, heads, n_tokens, head_dim, block_size, top_n, window_blocks,
+                                 abi.BSA_BF16 if dtype == torch.bfloat16 else abi.BSA_F32, scale)
+        self.shape = (batch, heads, n_tokens, head_dim)
+        self.dtype = dtype
+        self.m = n_tokens // block_size
+        self.workspace_bytes = abi.bsa_workspace_size(self.cfg)
+        self.workspace = torch.zeros(self.workspace_bytes, dtype=torch.uint8, device=device)
+        self.sel_idx = torch.empty((batch, heads, self.m, top_n), dtype=torch.int32, device=device)
+
+    @classmethod
+    def from_config(cls, cfg, device="cuda", scale: float = 0.0) -> "BSA":
+        return cls(cfg.batch, cfg.heads, cfg.n_tokens, cfg.head_dim, cfg.block_size, cfg.top_n,
+                   cfg.window_blocks, torch.bfloat16 if cfg.dtype == "bf16" else torch.float32, scale,
+                   device)
+
+    def __call__(self, q, k, v, gates, out=None) -> torch.Tensor:
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            _require(t, name, self.dtype, self.shape)
+        _require(gates, "gates", torch.float32, self.shape[:3] + (3,))
+        if out is None:
+            out = torch.empty_like(q)
+        _require(out, "out", self.dtype, self.shape)
+        abi.bsa_forward(self.cfg, q, k, v, gates, out, self.sel_idx, self.workspace, self.workspace_bytes)
+        return out
+
+    def check_status(self) -> int:
+        """Synchronise and return the kernels' status code (0 = OK); resets it."""
+        return abi.bsa_check_status(self.workspace)
+
+
+def forward(q, k, v, gates, block_size: int, top_n: int, window_blocks: int = 1, scale: float = 0.0,
+            return_indices: bool = False):
+    """One-shot BSA forward (allocates a workspace; use BSA for repeated calls)."""
+    b, h, n, d = q.shape
+    bsa = BSA(b, h, n, d, block_size, top_n, window_blocks, q.dtype, scale, q.device)
+    out = bsa(q, k, v, gates)
+    return (out, bsa.sel_idx) if return_indices else out
+
+
+def pool(q, k, v, block_size: int):
+    """Block means of q, k, v -> three float32 tensors [B, H, m, d]."""
+    b, h, n, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require(t, name, q.dtype, q.shape)
+    cfg = config_for(q, block_size, 1, 0)
+    outs = [torch.empty((b, h, n // block_size, d), dtype=torch.float32, device=q.device) for _ in range(3)]
+    abi.bsa_pool(cfg, q, k, v, *outs)
+    return tuple(outs)
+
+
+def compress_select(qbar, kbar, vbar, top_n: int, block_size: int, dtype=torch.bfloat16,
+                    scale: float = 0.0):
+    """Compressed branch + top-n from pooled tensors -> (o_cg_block [B,H,m,d], sel_idx [B,H,m,n])."""
+    b, h, m, d = qbar.shape
+    for name, t in (("qbar", qbar), ("kbar", kbar), ("vbar", vbar)):
+        _require(t, name, torch.float32, qbar.shape)
+    cfg = abi.BsaConfig(b, h, m * block_size, d, block_size, top_n, 0,
+                        abi.BSA_BF16 if dtype == torch.bfloat16 else abi.BSA_F32, scale)
+    o_cg = torch.empty_like(qbar)
+    idx = torch.empty((b, h, m, top_n), dtype=torch.int32, device=qbar.device)
+    abi.bsa_compress_select(cfg, qbar, kbar, vbar, o_cg, idx)
+    return o_cg, idx
+
+
+def fine_attention(q, k, v, gates, o_cg_block, sel_idx, block_size: int, window_blocks: int = 1,
+                   scale: float = 0.0, status_word=None, out=None):
+    """Selection + local branches and gated combine from given o_cg_block and sel_idx."""
+    b, h, n, d = q.shape
+    top_n = sel_idx.shape[-1]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require(t, name, q.dtype, q.shape)
+    _require(gates, "gates", torch.float32, (b, h, n, 3))
+    _require(o_cg_block, "o_cg_block", torch.float32, (b, h, n // block_size, d))
+    _require(sel_idx, "sel_idx", torch.int32, (b, h, n // block_size, top_n))
+    cfg = config_for(q, block_size, top_n, window_blocks, scale)
+    if out is None:
+        out = torch.empty_like(q)
+    abi.bsa_fine_attention(cfg, q, k, v, gates, o_cg_block, sel_idx, out, status_word)
+    return out

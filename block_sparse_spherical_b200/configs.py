@@ -25,10 +25,11 @@ class BSAConfig:
     window_blocks: int
     dtype: str  # "f32" or "bf16"
     seed: int
+    tokens: int = 0  # explicit N for non-HEALPix test shapes; 0 means 12 * nside**2
 
     @property
     def n_tokens(self) -> int:
-        return 12 * self.nside * self.nside
+        return self.tokens if self.tokens else 12 * self.nside * self.nside
 
     @property
     def n_blocks(self) -> int:

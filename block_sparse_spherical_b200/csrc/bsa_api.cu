@@ -1,0 +1,189 @@
+// C ABI of the BSA forward pass (declared in include/bsa.h): argument
+// validation, workspace layout and kernel dispatch. No allocation, no
+// synchronisation (except bsa_check_status), no global state.
+#include <math.h>
+#include <stdint.h>
+
+#include "bsa_internal.cuh"
+
+namespace {
+
+using bsa::Problem;
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+bool shape_supported(int32_t dtype, int32_t bk, int32_t d) {
+    return (dtype == BSA_BF16 && bk == 64 && d == 64) || (dtype == BSA_F32 && bk == 64 && d == 64) ||
+           (dtype == BSA_F32 && bk == 16 && d == 32);
+}
+
+bsa_status make_problem(const bsa_config *cfg, Problem *p) {
+    if (!cfg) return BSA_ERR_INVALID_ARG;
+    if (cfg->batch < 1 || cfg->heads < 1 || cfg->n_tokens < 1 || cfg->head_dim < 1 || cfg->block_size < 1)
+        return BSA_ERR_INVALID_ARG;
+    if (cfg->n_tokens % cfg->block_size != 0) return BSA_ERR_INVALID_ARG;
+    const int64_t m = cfg->n_tokens / cfg->block_size;
+    if (cfg->top_n < 1 || cfg->top_n > m || cfg->window_blocks < 0) return BSA_ERR_INVALID_ARG;
+    if (cfg->dtype != BSA_F32 && cfg->dtype != BSA_BF16) return BSA_ERR_INVALID_ARG;
+    if (!(cfg->scale >= 0.0f) || isinf(cfg->scale)) return BSA_ERR_INVALID_ARG;
+    if (!shape_supported(cfg->dtype, cfg->block_size, cfg->head_dim)) return BSA_ERR_UNSUPPORTED;
+    if (cfg->top_n > bsa::kMaxTopN) return BSA_ERR_UNSUPPORTED;
+    const int64_t slabs = (int64_t)cfg->batch * cfg->heads;
+    if (slabs > 65535) return BSA_ERR_UNSUPPORTED;            // grid.y of the per-slab kernels
+    p->batch = cfg->batch;
+    p->heads = cfg->heads;
+    p->n_tokens = cfg->n_tokens;
+    p->head_dim = cfg->head_dim;
+    p->block_size = cfg->block_size;
+    p->top_n = cfg->top_n;
+    p->window = cfg->window_blocks;
+    p->m = m;
+    p->slabs = slabs;
+    p->dtype = (bsa_dtype)cfg->dtype;
+    p->scale = cfg->scale > 0.0f ? cfg->scale : 1.0f / sqrtf((float)cfg->head_dim);
+    return BSA_OK;
+}
+
+struct WorkspaceLayout {
+    size_t status, qbar, kbar, vbar, o_cg, idx, total;
+};
+
+WorkspaceLayout layout_of(const Problem &p) {
+    const size_t pooled = (size_t)p.slabs * p.m * p.head_dim * sizeof(float);
+    const size_t idx = (size_t)p.slabs * p.m * p.top_n * sizeof(int32_t);
+    WorkspaceLayout w;
+    w.status = 0;
+    w.qbar = kAlign;
+    w.kbar = w.qbar + round_up(pooled);
+    w.vbar = w.kbar + round_up(pooled);
+    w.o_cg = w.vbar + round_up(pooled);
+    w.idx = w.o_cg + round_up(pooled);
+    w.total = w.idx + round_up(idx);
+    return w;
+}
+
+bsa_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return BSA_OK;
+    if (e == cudaErrorNotSupported) return BSA_ERR_UNSUPPORTED;
+    return BSA_ERR_CUDA;
+}
+
+cudaError_t launch_fine(const Problem &p, const void *q, const void *k, const void *v,
+                        const float *gates, const float *o_cg, const int32_t *idx, void *out,
+                        uint32_t *status, cudaStream_t stream) {
+    cudaError_t e = bsa::launch_attend_tc(p, q, k, v, gates, o_cg, idx, out, status, stream);
+    if (e != cudaErrorNotSupported) return e;
+    return bsa::launch_attend_simt(p, q, k, v, gates, o_cg, idx, out, status, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+bsa_status bsa_pool(const bsa_config *cfg, const void *q, const void *k, const void *v,
+                    float *qbar, float *kbar, float *vbar, cudaStream_t stream) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (!q || !k || !v || !qbar || !kbar || !vbar) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(qbar) || !aligned16(kbar) ||
+        !aligned16(vbar))
+        return BSA_ERR_ALIGNMENT;
+    return from_cuda(bsa::launch_pool(p, q, k, v, qbar, kbar, vbar, stream));
+}
+
+bsa_status bsa_compress_select(const bsa_config *cfg, const float *qbar, const float *kbar,
+                               const float *vbar, float *o_cg_block, int32_t *sel_idx,
+                               cudaStream_t stream) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (!qbar || !kbar || !vbar || !o_cg_block || !sel_idx) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(qbar) || !aligned16(kbar) || !aligned16(vbar) || !aligned16(o_cg_block) ||
+        !aligned16(sel_idx))
+        return BSA_ERR_ALIGNMENT;
+    return from_cuda(bsa::launch_compress_select(p, qbar, kbar, vbar, o_cg_block, sel_idx, stream));
+}
+
+bsa_status bsa_fine_attention(const bsa_config *cfg, const void *q, const void *k, const void *v,
+                              const float *gates, const float *o_cg_block, const int32_t *sel_idx,
+                              void *out, uint32_t *status_word, cudaStream_t stream) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (!q || !k || !v || !gates || !o_cg_block || !sel_idx || !out) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gates) || !aligned16(o_cg_block) ||
+        !aligned16(sel_idx) || !aligned16(out) || ((uintptr_t)status_word & 3u))
+        return BSA_ERR_ALIGNMENT;
+    return from_cuda(launch_fine(p, q, k, v, gates, o_cg_block, sel_idx, out, status_word, stream));
+}
+
+bsa_status bsa_workspace_size(const bsa_config *cfg, size_t *bytes) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (!bytes) return BSA_ERR_INVALID_ARG;
+    *bytes = layout_of(p).total;
+    return BSA_OK;
+}
+
+bsa_status bsa_forward(const bsa_config *cfg, const void *q, const void *k, const void *v,
+                       const float *gates, void *out, int32_t *sel_idx_out, void *workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (!q || !k || !v || !gates || !out) return BSA_ERR_INVALID_ARG;
+    if (!workspace) return BSA_ERR_WORKSPACE;
+    const WorkspaceLayout L = layout_of(p);
+    if (workspace_bytes < L.total) return BSA_ERR_WORKSPACE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gates) || !aligned16(out) ||
+        !aligned16(sel_idx_out) || ((uintptr_t)workspace & (kAlign - 1)))
+        return BSA_ERR_ALIGNMENT;
+    char *ws = static_cast<char *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws + L.status);
+    float *qbar = reinterpret_cast<float *>(ws + L.qbar);
+    float *kbar = reinterpret_cast<float *>(ws + L.kbar);
+    float *vbar = reinterpret_cast<float *>(ws + L.vbar);
+    float *ocg = reinterpret_cast<float *>(ws + L.o_cg);
+    int32_t *idx = sel_idx_out ? sel_idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
+    cudaError_t e = bsa::launch_pool(p, q, k, v, qbar, kbar, vbar, stream);
+    if (e == cudaSuccess) e = bsa::launch_compress_select(p, qbar, kbar, vbar, ocg, idx, stream);
+    if (e == cudaSuccess) e = launch_fine(p, q, k, v, gates, ocg, idx, out, status, stream);
+    return from_cuda(e);
+}
+
+bsa_status bsa_check_status(const void *status_word, cudaStream_t stream) {
+    if (!status_word || ((uintptr_t)status_word & 3u)) return BSA_ERR_INVALID_ARG;
+    uint32_t word = 0;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return BSA_ERR_CUDA;
+    if (cudaMemcpy(&word, status_word, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return BSA_ERR_CUDA;
+    if (word != 0) {
+        if (cudaMemsetAsync(const_cast<void *>(status_word), 0, sizeof(word), stream) != cudaSuccess ||
+            cudaStreamSynchronize(stream) != cudaSuccess)
+            return BSA_ERR_CUDA;
+    }
+    if (word & bsa::kStatusTimeout) return BSA_ERR_TIMEOUT;
+    if (word & bsa::kStatusBadIndex) return BSA_ERR_INDEX;
+    return BSA_OK;
+}
+
+const char *bsa_status_string(bsa_status s) {
+    switch (s) {
+        case BSA_OK: return "BSA_OK";
+        case BSA_ERR_INVALID_ARG: return "BSA_ERR_INVALID_ARG: invalid argument";
+        case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED: shape or dtype not compiled";
+        case BSA_ERR_ALIGNMENT: return "BSA_ERR_ALIGNMENT: pointer not 16-byte aligned";
+        case BSA_ERR_CUDA: return "BSA_ERR_CUDA: CUDA runtime or launch failure";
+        case BSA_ERR_TIMEOUT: return "BSA_ERR_TIMEOUT: a kernel's bounded wait expired";
+        case BSA_ERR_WORKSPACE: return "BSA_ERR_WORKSPACE: workspace missing or too small";
+        case BSA_ERR_INDEX: return "BSA_ERR_INDEX: block index outside [0, m)";
+    }
+    return "BSA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

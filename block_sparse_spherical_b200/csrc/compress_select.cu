@@ -1,0 +1,323 @@
+// Compressed branch (a) and top-n block selection of branch (b), BSA section
+// of the MOSAIC note, in fp32 on the CUDA cores:
+//
+//   z_ij = s·q̄_i·k̄_j,   o_cg_i = Σ_j softmax_j(z_ij) v̄_j,
+//   sel_i = top-n blocks j by (z_ij desc, j asc).
+//
+// One CTA owns 64 query blocks (rows) of one slab and streams the slab's k̄/v̄
+// in tiles of 64 key blocks through shared memory (cp.async, double
+// buffered). Per tile it forms the 64x64 logit tile in registers, runs one
+// online-softmax step, merges the tile into every row's running top-n list,
+// and accumulates P·v̄. The m×m logit matrix never leaves the SM.
+//
+// Thread layout (256 threads): warp w, half h = lane/16, tx = lane%16,
+// ty = 2w+h. Thread (ty,tx) owns rows 4ty..4ty+3; its logit columns are
+// tx+16jj (jj<4) and its output columns are tx*(D/16)..+D/16. A row is thus
+// owned by the 16 lanes of one half-warp, which also hold that row's sorted
+// top-n list (entry e = tx + 16*slot) and update it with shuffles only.
+#include <math_constants.h>
+
+#include "bsa_internal.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int BM = 64;        // query blocks per CTA
+constexpr int BN = 64;        // key blocks per tile
+constexpr int LDS = 68;       // padded smem row stride (floats) for 64-wide tiles
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool valid) {
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    const int bytes = valid ? 16 : 0;   // 0 => zero fill
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N));
+}
+
+// (av, ai) ranks above (bv, bi): larger logit, or equal logit and lower index.
+__device__ __forceinline__ bool ranks_above(float av, int ai, float bv, int bi) {
+    return av > bv || (av == bv && ai < bi);
+}
+
+template <int D>
+__device__ __forceinline__ void load_rows(float *dst, const float *src, int row0, int m, int tid) {
+    // BM rows x D floats -> dst[r*LDS + c], rows >= m zero filled
+    constexpr int CPR = D / 4;                 // 16-byte chunks per row
+    constexpr int TOTAL = BM * CPR;
+#pragma unroll
+    for (int c = tid; c < TOTAL; c += 256) {
+        const int r = c / CPR, col = (c % CPR) * 4;
+        const bool ok = row0 + r < m;
+        const float *g = src + (int64_t)(ok ? row0 + r : 0) * D + col;
+        cp_async16(dst + r * LDS + col, g, ok);
+    }
+}
+
+template <int D, int NPL>
+__global__ void __launch_bounds__(256, 2)
+compress_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar,
+                       const float *__restrict__ vbar, float *__restrict__ o_cg,
+                       int32_t *__restrict__ idx_out, int m, int n, float scale_log2) {
+    static_assert(D == 32 || D == 64, "head_dim 32 or 64");
+    constexpr int DPT = D / 16;                // output columns per thread
+    extern __shared__ __align__(16) float smem[];
+    float *Qs = smem;                          // [BM][LDS]
+    float *Ks = Qs + BM * LDS;                 // [2][BN][LDS]
+    float *Vs = Ks + 2 * BN * LDS;             // [2][BN][LDS]
+    float *Ps = Vs + 2 * BN * LDS;             // [BM][LDS]
+
+    const int tid = threadIdx.x, lane = tid & 31, half = lane >> 4, tx = lane & 15;
+    const int ty = 2 * (tid >> 5) + half;
+    const int row0 = blockIdx.x * BM;
+    const int64_t slab = blockIdx.y;
+    const float *q = qbar + slab * (int64_t)m * D;
+    const float *k = kbar + slab * (int64_t)m * D;
+    const float *v = vbar + slab * (int64_t)m * D;
+
+    load_rows<D>(Qs, q, row0, m, tid);
+    load_rows<D>(Ks, k, 0, m, tid);
+    load_rows<D>(Vs, v, 0, m, tid);
+    cp_async_commit();
+
+    float o[4][DPT];
+    float mrun[4], lrun[4];
+    float lv[4][NPL];
+    int li[4][NPL];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        mrun[i] = -CUDART_INF_F;
+        lrun[i] = 0.f;
+#pragma unroll
+        for (int c = 0; c < DPT; ++c) o[i][c] = 0.f;
+#pragma unroll
+        for (int h = 0; h < NPL; ++h) { lv[i][h] = -CUDART_INF_F; li[i][h] = 0x7fffffff; }
+    }
+    // the list's n-th entry (the admission threshold) lives at lane tn, slot hn
+    const int tn = (n - 1) & 15, hn = (n - 1) >> 4;
+    const unsigned FULL = 0xffffffffu;
+    const int ntiles = (m + BN - 1) / BN;
+
+    for (int t = 0; t < ntiles; ++t) {
+        const int buf = t & 1;
+        if (t + 1 < ntiles) {
+            load_rows<D>(Ks + (buf ^ 1) * BN * LDS, k, (t + 1) * BN, m, tid);
+            load_rows<D>(Vs + (buf ^ 1) * BN * LDS, v, (t + 1) * BN, m, tid);
+        }
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        const float *Kt = Ks + buf * BN * LDS;
+        const float *Vt = Vs + buf * BN * LDS;
+        const int col0 = t * BN;
+
+        // ---- logits of the tile: s[i][jj] for row 4ty+i, key col0+tx+16jj
+        float s[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) s[i][jj] = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < D; c += 4) {
+            float4 qa[4], kb[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) qa[i] = *reinterpret_cast<const float4 *>(Qs + (4 * ty + i) * LDS + c);
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) kb[jj] = *reinterpret_cast<const float4 *>(Kt + (tx + 16 * jj) * LDS + c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    s[i][jj] = fmaf(qa[i].x, kb[jj].x, s[i][jj]);
+                    s[i][jj] = fmaf(qa[i].y, kb[jj].y, s[i][jj]);
+                    s[i][jj] = fmaf(qa[i].z, kb[jj].z, s[i][jj]);
+                    s[i][jj] = fmaf(qa[i].w, kb[jj].w, s[i][jj]);
+                }
+        }
+        // log2-domain logits; columns past m do not exist
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+            const bool ok = col0 + tx + 16 * jj < m;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s[i][jj] = ok ? s[i][jj] * scale_log2 : -CUDART_INF_F;
+        }
+
+        // ---- top-n merge (rows of this half-warp), candidates in any order
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float tv = -CUDART_INF_F;
+            int ti = 0x7fffffff;
+#pragma unroll
+            for (int h = 0; h < NPL; ++h)
+                if (h == hn) { tv = lv[i][h]; ti = li[i][h]; }
+            tv = __shfl_sync(FULL, tv, tn, 16);
+            ti = __shfl_sync(FULL, ti, tn, 16);
+            unsigned cand = 0;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int j = col0 + tx + 16 * jj;
+                if (j < m && ranks_above(s[i][jj], j, tv, ti)) cand |= 1u << jj;
+            }
+            while (__any_sync(FULL, cand != 0)) {
+                const unsigned ball = __ballot_sync(FULL, cand != 0);
+                const unsigned mine = (ball >> (16 * half)) & 0xffffu;
+                const int leader = mine ? (__ffs(mine) - 1) : 0;
+                const int jj = cand ? (__ffs(cand) - 1) : 0;
+                float my_s = s[i][0];
+#pragma unroll
+                for (int u = 1; u < 4; ++u)
+                    if (jj == u) my_s = s[i][u];
+                float cs = __shfl_sync(FULL, my_s, leader, 16);
+                const int cj = __shfl_sync(FULL, col0 + tx + 16 * jj, leader, 16);
+                if (!mine) cs = -CUDART_INF_F;         // this half has nothing to insert
+                if (mine && tx == leader) cand &= cand - 1;
+                // position of the candidate = number of entries ranking above it
+                int pos = 0;
+#pragma unroll
+                for (int h = 0; h < NPL; ++h) {
+                    const unsigned ab = __ballot_sync(FULL, ranks_above(lv[i][h], li[i][h], cs, cj));
+                    pos += __popc((ab >> (16 * half)) & 0xffffu);
+                }
+                const bool insert = mine && pos < n;
+                // shift entries >= pos down by one (slots high to low read old values)
+#pragma unroll
+                for (int h = NPL - 1; h >= 0; --h) {
+                    float upv = __shfl_up_sync(FULL, lv[i][h], 1, 16);
+                    int upi = __shfl_up_sync(FULL, li[i][h], 1, 16);
+                    if (h > 0) {
+                        const float pv = __shfl_sync(FULL, lv[i][h - 1], 15, 16);
+                        const int pi = __shfl_sync(FULL, li[i][h - 1], 15, 16);
+                        if (tx == 0) { upv = pv; upi = pi; }
+                    }
+                    const int e = tx + 16 * h;
+                    if (insert && e >= pos) {
+                        if (e == pos) { lv[i][h] = cs; li[i][h] = cj; }
+                        else { lv[i][h] = upv; li[i][h] = upi; }
+                    }
+                }
+                // refresh the threshold and drop candidates that no longer qualify
+                float nv = -CUDART_INF_F;
+                int ni = 0x7fffffff;
+#pragma unroll
+                for (int h = 0; h < NPL; ++h)
+                    if (h == hn) { nv = lv[i][h]; ni = li[i][h]; }
+                nv = __shfl_sync(FULL, nv, tn, 16);
+                ni = __shfl_sync(FULL, ni, tn, 16);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if ((cand >> u & 1u) && !ranks_above(s[i][u], col0 + tx + 16 * u, nv, ni)) cand &= ~(1u << u);
+            }
+        }
+
+        // ---- online softmax step
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float mx = fmaxf(fmaxf(s[i][0], s[i][1]), fmaxf(s[i][2], s[i][3]));
+#pragma unroll
+            for (int off = 1; off < 16; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, off));
+            const float mnew = fmaxf(mrun[i], mx);
+            const float alpha = exp2f(mrun[i] - mnew);   // 0 on the first tile
+            mrun[i] = mnew;
+            float ls = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const float pexp = exp2f(s[i][jj] - mnew);
+                ls += pexp;
+                Ps[(4 * ty + i) * LDS + tx + 16 * jj] = pexp;
+            }
+            lrun[i] = lrun[i] * alpha + ls;
+#pragma unroll
+            for (int c = 0; c < DPT; ++c) o[i][c] *= alpha;
+        }
+        __syncthreads();
+
+        // ---- o += P · v̄_tile
+#pragma unroll 4
+        for (int j = 0; j < BN; j += 4) {
+            float4 pa[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pa[i] = *reinterpret_cast<const float4 *>(Ps + (4 * ty + i) * LDS + j);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float vv[DPT];
+                if constexpr (DPT == 4) {
+                    const float4 t4 = *reinterpret_cast<const float4 *>(Vt + (j + u) * LDS + tx * 4);
+                    vv[0] = t4.x; vv[1] = t4.y; vv[2] = t4.z; vv[3] = t4.w;
+                } else {
+                    const float2 t2 = *reinterpret_cast<const float2 *>(Vt + (j + u) * LDS + tx * 2);
+                    vv[0] = t2.x; vv[1] = t2.y;
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float pu = u == 0 ? pa[i].x : u == 1 ? pa[i].y : u == 2 ? pa[i].z : pa[i].w;
+#pragma unroll
+                    for (int c = 0; c < DPT; ++c) o[i][c] = fmaf(pu, vv[c], o[i][c]);
+                }
+            }
+        }
+        __syncthreads();   // Ps and this K/V buffer are rewritten next
+    }
+
+    // ---- finish: normalise, write o_cg and the index lists
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float l = lrun[i];
+#pragma unroll
+        for (int off = 1; off < 16; off <<= 1) l += __shfl_xor_sync(FULL, l, off);
+        const int r = row0 + 4 * ty + i;
+        if (r < m) {
+            const float inv = 1.0f / l;
+            float *dst = o_cg + (slab * m + r) * (int64_t)D + tx * DPT;
+            if constexpr (DPT == 4)
+                *reinterpret_cast<float4 *>(dst) = make_float4(o[i][0] * inv, o[i][1] * inv, o[i][2] * inv, o[i][3] * inv);
+            else
+                *reinterpret_cast<float2 *>(dst) = make_float2(o[i][0] * inv, o[i][1] * inv);
+            int32_t *ix = idx_out + (slab * m + r) * (int64_t)n;
+#pragma unroll
+            for (int h = 0; h < NPL; ++h) {
+                const int e = tx + 16 * h;
+                if (e < n) ix[e] = li[i][h];
+            }
+        }
+    }
+}
+
+template <int D, int NPL>
+cudaError_t launch(const Problem &p, const float *qb, const float *kb, const float *vb, float *ocg,
+                   int32_t *idx, cudaStream_t s) {
+    const size_t smem = (size_t)(BM * LDS + 4 * BN * LDS + BM * LDS) * sizeof(float);
+    auto kern = compress_select_kernel<D, NPL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)((p.m + BM - 1) / BM), (unsigned)p.slabs);
+    const float scale_log2 = p.scale * 1.4426950408889634f;
+    kern<<<grid, 256, smem, s>>>(qb, kb, vb, ocg, idx, (int)p.m, (int)p.top_n, scale_log2);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_compress_select(const Problem &p, const float *qbar, const float *kbar,
+                                   const float *vbar, float *o_cg, int32_t *idx,
+                                   cudaStream_t stream) {
+    if (p.top_n > kMaxTopN) return cudaErrorNotSupported;
+    const int npl = (int)((p.top_n + 15) / 16);
+    if (p.head_dim == 64) {
+        switch (npl) {
+            case 1: return launch<64, 1>(p, qbar, kbar, vbar, o_cg, idx, stream);
+            case 2: return launch<64, 2>(p, qbar, kbar, vbar, o_cg, idx, stream);
+            default: return launch<64, 4>(p, qbar, kbar, vbar, o_cg, idx, stream);
+        }
+    }
+    if (p.head_dim == 32) {
+        switch (npl) {
+            case 1: return launch<32, 1>(p, qbar, kbar, vbar, o_cg, idx, stream);
+            case 2: return launch<32, 2>(p, qbar, kbar, vbar, o_cg, idx, stream);
+            default: return launch<32, 4>(p, qbar, kbar, vbar, o_cg, idx, stream);
+        }
+    }
+    return cudaErrorNotSupported;
+}
+
+}  // namespace bsa

@@ -1,0 +1,108 @@
+"""The C-ABI library without a GPU: it loads, exports every declared symbol,
+and rejects bad arguments on the host before any launch (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_spherical_b200 import abi, build
+from block_sparse_spherical_b200.configs import CONFIGS
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "bsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return abi.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"BSA_API\s+[\w\s\*]+?\b(bsa_\w+)\s*\(", src)
+
+
+def test_header_declares_the_binding_names():
+    names = declared_functions()
+    assert sorted(names) == sorted(abi.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in abi.STATUS_NAMES.items():
+        assert abi.bsa_status_string(code).startswith(name)
+    assert "UNKNOWN" in abi.bsa_status_string(99)
+
+
+def cfg_of(**over):
+    c = abi.make_config(CONFIGS["nside32"])
+    for k, v in over.items():
+        setattr(c, k, v)
+    return c
+
+
+def ws_size(c):
+    n = ctypes.c_size_t(0)
+    return abi.load().bsa_workspace_size(ctypes.byref(c), ctypes.byref(n)), n.value
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(batch=0), 1), (dict(heads=-1), 1), (dict(n_tokens=0), 1), (dict(head_dim=0), 1),
+    (dict(block_size=0), 1), (dict(n_tokens=12289), 1), (dict(top_n=0), 1), (dict(top_n=193), 1),
+    (dict(window_blocks=-1), 1), (dict(dtype=7), 1), (dict(scale=-1.0), 1), (dict(scale=float("nan")), 1),
+    (dict(scale=float("inf")), 1),
+    (dict(head_dim=128), 2), (dict(block_size=32), 2), (dict(dtype=0, block_size=16, head_dim=64), 2),
+    (dict(top_n=65), 2), (dict(batch=70000), 2),
+])
+def test_workspace_size_validation(lib, over, code):
+    rc, _ = ws_size(cfg_of(**over))
+    assert rc == code
+
+
+def test_workspace_size_layout(lib):
+    for cfg in CONFIGS.values():
+        c = abi.make_config(cfg)
+        rc, n = ws_size(c)
+        assert rc == 0
+        pooled = cfg.slabs * cfg.n_blocks * cfg.head_dim * 4
+        idx = cfg.slabs * cfg.n_blocks * cfg.top_n * 4
+        up = lambda x: (x + 255) // 256 * 256
+        assert n == 256 + 4 * up(pooled) + up(idx)
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch(lib):
+    c = abi.make_config(CONFIGS["nside32"])
+    L = abi.load()
+    cp = ctypes.byref(c)
+    A = 4096          # never dereferenced: validation fails first
+    # null pointers
+    assert L.bsa_pool(cp, None, A, A, A, A, A, None) == 1
+    assert L.bsa_compress_select(cp, A, A, A, A, None, None) == 1
+    assert L.bsa_fine_attention(cp, A, A, A, A, A, A, None, None, None) == 1
+    assert L.bsa_forward(cp, A, A, A, None, A, None, A, 1 << 30, None) == 1
+    assert L.bsa_check_status(None, None) == 1
+    # misalignment
+    assert L.bsa_pool(cp, A + 2, A, A, A, A, A, None) == 3
+    assert L.bsa_compress_select(cp, A, A, A + 8, A, A, None) == 3
+    assert L.bsa_fine_attention(cp, A, A, A, A, A, A, A, A + 2, None) == 3
+    assert L.bsa_forward(cp, A, A, A, A, A, None, A + 16, 1 << 30, None) == 3
+    # workspace missing / too small
+    assert L.bsa_forward(cp, A, A, A, A, A, None, None, 1 << 30, None) == 6
+    _, need = ws_size(c)
+    assert L.bsa_forward(cp, A, A, A, A, A, None, A, need - 1, None) == 6
+    # bad config with good pointers
+    bad = cfg_of(top_n=0)
+    assert L.bsa_forward(ctypes.byref(bad), A, A, A, A, A, None, A, need, None) == 1
+    assert L.bsa_pool(None, A, A, A, A, A, A, None) == 1
+
+
+def test_python_binding_raises_on_error(lib):
+    c = cfg_of(top_n=0)
+    with pytest.raises(abi.BsaError) as e:
+        abi.bsa_workspace_size(c)
+    assert e.value.code == 1

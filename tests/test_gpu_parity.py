@@ -1,0 +1,120 @@
+"""CUDA path vs the fp64 oracle on the seeded workloads (needs a B200).
+
+Small workloads are checked everywhere; the large ones (Nside 64/128/256)
+run at full size in the same launch configuration as the benchmark and are
+checked on sampled slabs and query-block ranges (head, middle, tail).
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_spherical_b200 import abi, api
+from block_sparse_spherical_b200.configs import CONFIGS
+
+import parity
+
+pytestmark = pytest.mark.gpu
+
+SAMPLING = {  # config -> (slabs to check, max query blocks per slab or None for all)
+    "tiny_nside8": (None, None),
+    "nside32": (None, None),
+    "nside64": ([0, 13, 31], 96),
+    "nside128": ([0, 31], 96),
+    "nside256": ([0, 7], 48),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    abi.load()
+
+
+def run_all(cfg):
+    q, k, v, g = parity.device_inputs(cfg)
+    qb, kb, vb = api.pool(q, k, v, cfg.block_size)
+    o_cg, idx = api.compress_select(qb, kb, vb, cfg.top_n, cfg.block_size,
+                                    torch.bfloat16 if cfg.dtype == "bf16" else torch.float32)
+    bsa = api.BSA.from_config(cfg)
+    out = bsa(q, k, v, g)
+    torch.cuda.synchronize()
+    assert bsa.check_status() == 0
+    assert torch.equal(bsa.sel_idx, idx), "bsa_forward chose other blocks than bsa_compress_select"
+    out2 = bsa(q, k, v, g)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2), "bsa_forward is not deterministic"
+    return dict(qbar=qb, kbar=kb, vbar=vb, o_cg=o_cg, idx=idx, out=out)
+
+
+@pytest.mark.parametrize("name", list(CONFIGS))
+def test_workload_parity(name):
+    cfg = CONFIGS[name]
+    res = run_all(cfg)
+    slabs, max_rows = SAMPLING[name]
+    slabs = range(cfg.slabs) if slabs is None else slabs
+    ties = 0
+    for s in slabs:
+        b, h = divmod(s, cfg.heads)
+        gpu = {key: parity.to_np(t[b, h]) for key, t in res.items()}
+        summ = parity.check_slab(cfg, s, gpu, max_rows)
+        ties += summ["near_ties"]
+    assert np.isfinite(parity.to_np(res["out"][0, 0])).all()
+    print(f"{name}: near-tie rows checked by the validity rule: {ties}")
+
+
+EDGE = {
+    # name: (block, d, dtype, tokens, batch, heads, top_n, window)
+    "single_block": (64, 64, "bf16", 64, 1, 1, 1, 1),
+    "two_blocks_all_selected_w0": (64, 64, "bf16", 128, 1, 2, 2, 0),
+    "ragged_m100": (64, 64, "bf16", 6400, 2, 3, 16, 1),
+    "ragged_m300_n64_w2": (64, 64, "bf16", 19200, 1, 2, 64, 2),
+    "window_covers_all": (64, 64, "bf16", 640, 1, 2, 3, 20),
+    "topn_equals_m": (64, 64, "bf16", 2048, 1, 2, 32, 1),
+    "f32_block64": (64, 64, "f32", 4096, 1, 2, 8, 1),
+    "f32_tiny_n_eq_m": (16, 32, "f32", 768, 1, 2, 48, 1),
+    "f32_tiny_ragged": (16, 32, "f32", 16 * 75, 3, 1, 5, 3),
+}
+
+
+@pytest.mark.parametrize("name", list(EDGE))
+def test_edge_cases(name):
+    bk, d, dt, tokens, b, h, n, w = EDGE[name]
+    cfg = CONFIGS["nside32"].with_(name=name, block_size=bk, head_dim=d, dtype=dt, tokens=tokens,
+                                   batch=b, heads=h, top_n=n, window_blocks=w, seed=100 + len(name))
+    res = run_all(cfg)
+    for s in range(cfg.slabs):
+        bi, hi = divmod(s, cfg.heads)
+        gpu = {key: parity.to_np(t[bi, hi]) for key, t in res.items()}
+        parity.check_slab(cfg, s, gpu, None)
+
+
+def test_bad_indices_are_flagged_not_followed():
+    cfg = CONFIGS["nside32"]
+    q, k, v, g = parity.device_inputs(cfg)
+    qb, kb, vb = api.pool(q, k, v, cfg.block_size)
+    o_cg, idx = api.compress_select(qb, kb, vb, cfg.top_n, cfg.block_size)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bad = idx.clone()
+    bad[0, 0, 0, 0] = -1
+    bad[0, 1, 5, 3] = cfg.n_blocks
+    out = api.fine_attention(q, k, v, g, o_cg, bad, cfg.block_size, cfg.window_blocks, status_word=status)
+    assert abi.bsa_check_status(status) == 7                # BSA_ERR_INDEX
+    assert abi.bsa_check_status(status) == 0                # reset by the first check
+    assert torch.isfinite(out.float()).all()
+    good = api.fine_attention(q, k, v, g, o_cg, idx, cfg.block_size, cfg.window_blocks, status_word=status)
+    assert abi.bsa_check_status(status) == 0
+    # rows without a bad index are unaffected
+    assert torch.equal(out[0, 2], good[0, 2])
+
+
+def test_binding_rejects_wrong_tensors():
+    cfg = CONFIGS["tiny_nside8"]
+    q, k, v, g = parity.device_inputs(cfg)
+    bsa = api.BSA.from_config(cfg)
+    with pytest.raises(TypeError):
+        bsa(q.to(torch.bfloat16), k, v, g)
+    with pytest.raises(ValueError):
+        bsa(q.transpose(2, 3), k, v, g)
+    with pytest.raises(ValueError):
+        bsa(q.cpu(), k, v, g)
