@@ -229,7 +229,7 @@ def run_ours(args, cfg, rank, world, local_rank):
 
     def host(a):
         t = torch.from_numpy(a)
-        return t.view(torch.bfloat16) if cfg.dtype == "bf16" else t
+        return t.view(torch.bfloat16) if a.dtype == np.uint16 else t
 
     q, k, v, g = (host(a).to(dev) for a in (qh, kh, vh, gh))
     stream = torch.cuda.current_stream(dev)
