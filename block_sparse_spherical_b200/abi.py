@@ -20,7 +20,7 @@ STATUS_NAMES = {
     4: "BSA_ERR_CUDA", 5: "BSA_ERR_TIMEOUT", 6: "BSA_ERR_WORKSPACE", 7: "BSA_ERR_INDEX",
 }
 EXPORTS = ("bsa_pool", "bsa_compress_select", "bsa_fine_attention", "bsa_workspace_size",
-           "bsa_forward", "bsa_check_status", "bsa_status_string")
+           "bsa_forward", "bsa_check_status", "bsa_status_string", "bsa_forward_noalloc")
 
 
 class BsaConfig(ctypes.Structure):
@@ -55,6 +55,7 @@ def load() -> ctypes.CDLL:
         "bsa_forward": [C, P, P, P, P, P, P, P, S, P],
         "bsa_check_status": [P, P],
         "bsa_status_string": [ctypes.c_int],
+        "bsa_forward_noalloc": [C, P, P, P, P, P, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -119,6 +120,14 @@ def bsa_forward(cfg: BsaConfig, q, k, v, gates, out, sel_idx_out, workspace, wor
     _check("bsa_forward", load().bsa_forward(
         ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(out), _ptr(sel_idx_out),
         _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def bsa_forward_noalloc(cfg: BsaConfig, q, k, v, gates, out, sel_idx_out=None, status_word=None,
+                        stream=None) -> None:
+    """bsa_forward without a caller workspace: the library's fixed 32 MiB device scratch is used."""
+    _check("bsa_forward_noalloc", load().bsa_forward_noalloc(
+        ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(out), _ptr(sel_idx_out),
+        _ptr(status_word), _stream(stream)))
 
 
 def bsa_check_status(status_word, stream=None) -> int:

@@ -187,3 +187,84 @@ const char *bsa_status_string(bsa_status s) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward pass.
+//
+// Some callers cannot call cudaMalloc at the point where they run BSA: code
+// that executes inside a host callback or another library's allocator hook,
+// plugins whose host framework owns every device allocation, or services
+// that must not touch the allocator on the request path. For them,
+// bsa_forward_noalloc runs the same three kernels as bsa_forward but keeps
+// the intermediates (pooled q̄/k̄/v̄, block-level compressed output, block
+// indices) in a fixed array of device memory that this library owns.
+//
+// The array lives in device global memory for as long as the library is
+// loaded, on every GPU that loads it, and is shared by every call on that
+// GPU: two calls whose work overlaps on the GPU (different streams, or
+// different host threads) race on it. Each call rewrites every byte it later
+// reads, so nothing in the array has to start at zero and leftovers of the
+// previous call are never used.
+// ---------------------------------------------------------------------------
+
+#include <mutex>
+
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB per GPU
+constexpr int kMaxDevices = 64;
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_bsa_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+
+std::once_flag g_scratch_once[kMaxDevices];
+void *g_scratch_ptr[kMaxDevices];
+cudaError_t g_scratch_err[kMaxDevices];
+
+// Device address of the scratch array on the current device. In host code
+// the array's name only stands in for it, so the address is looked up once
+// per device, with that device current, on the first call made there.
+cudaError_t noalloc_scratch(void **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::call_once(g_scratch_once[dev], [dev] {
+        void *p = nullptr;
+        g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_bsa_noalloc_scratch);
+        g_scratch_ptr[dev] = p;
+    });
+    if (g_scratch_err[dev] != cudaSuccess) return g_scratch_err[dev];
+    if (!g_scratch_ptr[dev]) return cudaErrorInvalidSymbol;
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" bsa_status bsa_forward_noalloc(const bsa_config *cfg, const void *q, const void *k, const void *v,
+                                          const float *gates, void *out, int32_t *sel_idx_out,
+                                          uint32_t *status_word, cudaStream_t stream) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (!q || !k || !v || !gates || !out) return BSA_ERR_INVALID_ARG;
+    const WorkspaceLayout L = layout_of(p);
+    if (L.total > kNoAllocScratchBytes) return BSA_ERR_WORKSPACE;   // problem too large for the fixed scratch
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gates) || !aligned16(out) ||
+        !aligned16(sel_idx_out) || ((uintptr_t)status_word & 3u))
+        return BSA_ERR_ALIGNMENT;
+    void *scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return BSA_ERR_CUDA;
+    char *ws = static_cast<char *>(scratch);
+    float *qbar = reinterpret_cast<float *>(ws + L.qbar);
+    float *kbar = reinterpret_cast<float *>(ws + L.kbar);
+    float *vbar = reinterpret_cast<float *>(ws + L.vbar);
+    float *ocg = reinterpret_cast<float *>(ws + L.o_cg);
+    int32_t *idx = sel_idx_out ? sel_idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
+    cudaError_t e = bsa::launch_pool(p, q, k, v, qbar, kbar, vbar, stream);
+    if (e == cudaSuccess) e = bsa::launch_compress_select(p, qbar, kbar, vbar, ocg, idx, stream);
+    if (e == cudaSuccess) e = launch_fine(p, q, k, v, gates, ocg, idx, out, status_word, stream);
+    return from_cuda(e);
+}

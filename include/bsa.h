@@ -133,6 +133,33 @@ BSA_API bsa_status bsa_forward(const bsa_config *cfg, const void *q, const void 
  */
 BSA_API bsa_status bsa_check_status(const void *status_word, cudaStream_t stream);
 
+/*
+ * Allocation-free variant of bsa_forward (the MOSAIC note has no counterpart:
+ * this is a deployment convenience, not a step of the method).
+ *
+ * For callers that cannot allocate device memory when they run BSA (code in
+ * a host callback or an allocator hook, plugins whose host framework owns all
+ * device allocations, request paths that must not touch the allocator). It
+ * runs the same three kernels as bsa_forward, but the intermediates live in
+ * a fixed 32 MiB array of device memory owned by the library instead of a
+ * caller workspace; the caller still passes q, k, v, gates and out (and the
+ * optional sel_idx_out / status_word, same meaning as in bsa_forward and
+ * bsa_fine_attention; status_word may be NULL).
+ *  - Returns BSA_ERR_WORKSPACE when bsa_workspace_size(cfg) exceeds 32 MiB
+ *    (e.g. Nside 64 with batch 4 x 8 heads fits; Nside 128 with 2 x 16 does not).
+ *  - Never calls cudaMalloc, cudaFree or any allocating routine.
+ *  - The array exists on every GPU that loads the library until the process
+ *    exits. The first call on each device looks up its device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls on a GPU share the array: calls that overlap on the GPU
+ *    (other streams, other host threads) race and must be serialised by the
+ *    caller. Each call rewrites everything it reads, so no part of the array
+ *    needs to start at zero.
+ */
+BSA_API bsa_status bsa_forward_noalloc(const bsa_config *cfg, const void *q, const void *k, const void *v,
+                                       const float *gates, void *out, int32_t *sel_idx_out,
+                                       uint32_t *status_word, cudaStream_t stream);
+
 /* Static, human-readable name of a status code. */
 BSA_API const char *bsa_status_string(bsa_status status);
 
