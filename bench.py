@@ -124,40 +124,63 @@ class ClockSampler:
 _SLAB_CACHE = {}
 
 
-def oracle_sample(cfg, target_s: float, slab: int = 0, lib=None):
-    """Time the oracle on a bounded sample of one slab; return (tokens/s, description, seconds)."""
-    import oracle
+def _slab64(cfg, slab):
     from block_sparse_spherical_b200.synthetic import make_slab
-    lib = lib or oracle.load()
     key = (cfg.name, slab)
     if key not in _SLAB_CACHE:
+        if len(_SLAB_CACHE) > 2:
+            _SLAB_CACHE.clear()
         s = make_slab(cfg, slab)
         _SLAB_CACHE[key] = tuple(x.astype(np.float64) for x in (s.q, s.k, s.v, s.gates))
-    q, k, v, g = _SLAB_CACHE[key]
+    return _SLAB_CACHE[key]
+
+
+def oracle_sample(cfg, target_s: float, lib=None):
+    """Time the oracle on a bounded sample of the workload; return (tokens/s, description, seconds).
+
+    Whole slabs (pool, compressed rows, selection+local+combine) are timed one
+    after another until about target_s seconds of oracle time are spent; the
+    last slab may be cut to its first query blocks (pooling pro-rated).
+    """
+    import oracle
+    lib = lib or oracle.load()
     bk, n, w, m = cfg.block_size, cfg.top_n, cfg.window_blocks, cfg.n_blocks
-    t0 = time.perf_counter()
-    qb, kb, vb = (oracle.pool(x, bk, lib=lib) for x in (q, k, v))
-    t_pool = time.perf_counter() - t0
-
-    def run(nblk):
-        t = time.perf_counter()
+    spent, tokens, slabs_done, part = 0.0, 0, 0, None
+    for slab in range(cfg.slabs):
+        q, k, v, g = _slab64(cfg, slab)
+        t0 = time.perf_counter()
+        qb, kb, vb = (oracle.pool(x, bk, lib=lib) for x in (q, k, v))
+        t_pool = time.perf_counter() - t0
+        left = target_s - spent
+        # estimate the per-block cost on a short probe, then size this slab's share
+        probe = min(m, 8)
+        t0 = time.perf_counter()
+        c = oracle.compressed_rows(qb, kb, vb, n, rows=(0, probe), lib=lib)
+        ocg = np.zeros((m, cfg.head_dim)); ocg[:probe] = c["o_cg"]
+        idx = np.zeros((m, n), np.int32); idx[:probe] = c["idx"]
+        oracle.fine_rows(q, k, v, g, ocg, idx, bk, n, w, qblocks=(0, probe), lib=lib)
+        t_probe = time.perf_counter() - t0
+        nblk = int(min(m, max(probe, probe * left / max(t_probe, 1e-6))))
+        t0 = time.perf_counter()
         c = oracle.compressed_rows(qb, kb, vb, n, rows=(0, nblk), lib=lib)
-        ocg = np.zeros((m, cfg.head_dim))
-        ocg[:nblk] = c["o_cg"]
-        idx = np.zeros((m, n), np.int32)
-        idx[:nblk] = c["idx"]
+        ocg = np.zeros((m, cfg.head_dim)); ocg[:nblk] = c["o_cg"]
+        idx = np.zeros((m, n), np.int32); idx[:nblk] = c["idx"]
         oracle.fine_rows(q, k, v, g, ocg, idx, bk, n, w, qblocks=(0, nblk), lib=lib)
-        return time.perf_counter() - t
-
-    probe = min(m, 8)
-    t_probe = run(probe)
-    nblk = int(min(m, max(probe, probe * target_s / max(t_probe, 1e-6))))
-    t_run = run(nblk) if nblk > probe else t_probe
-    elapsed = t_run + t_pool * nblk / m
-    tokens = nblk * bk
-    desc = (f"slab {slab} of {cfg.name}: query blocks 0..{nblk - 1} ({tokens} tokens; compressed rows "
-            f"over all {m} key blocks, selection+local+combine), pooling of the slab pro-rated by {nblk}/{m}")
-    return tokens / elapsed, desc, elapsed
+        spent += time.perf_counter() - t0 + t_pool * nblk / m
+        tokens += nblk * bk
+        if nblk < m:
+            part = nblk
+            break
+        slabs_done += 1
+        if spent >= target_s:
+            break
+    desc = f"{slabs_done} whole slab(s) of {cfg.name}"
+    if part is not None:
+        desc += f" + query blocks 0..{part - 1} of the next ({tokens} tokens in all; its pooling pro-rated)"
+    else:
+        desc += f" ({tokens} tokens)"
+    desc += "; each slab: pooling, compressed rows over all key blocks with top-n, selection+local+combine"
+    return tokens / spent, desc, spent
 
 
 def omp_threads():

@@ -1,9 +1,630 @@
-// Tensor-core (tcgen05 + TMEM + TMA) selection+local attention: not yet built.
+// Selection branch (b), local branch (c) and the gated combine of the BSA
+// section (MOSAIC note) on the sm_100a tensor cores: bf16 inputs, block 64,
+// head_dim 64, fp32 accumulation in tensor memory.
+//
+// Thanks to the NESTED order every key/value block is one contiguous 8 KB
+// span, so each is a single TMA box (64 rows x 128 B, 128-byte swizzle)
+// copied straight into the layout tcgen05.mma reads. Per query block the
+// kernel streams its 2w+1 local blocks and then its n selected blocks; for
+// each block it runs S = Q·Kᵀ (tcgen05.mma, M=64 N=64 K=64) into TMEM, an
+// online softmax on the CUDA cores, and O += P·V (tcgen05.mma, P from shared
+// memory). The local branch's output is folded into a register accumulator
+// together with the compressed branch (acc = g_CG·o_CG + g_L·o_L) before the
+// selection branch reuses the same TMEM accumulator; the epilogue adds
+// g_FG·o_FG and stores bf16.
+//
+// Organisation: a persistent grid of one CTA per SM, 384 threads, two
+// independent pipelines ("slots") per CTA. A slot works on a pair of
+// neighbouring query blocks (A, B) at a time; their M=64 accumulators live
+// in TMEM lanes 0-15 of each 32-lane sub-partition at adjacent 64-column
+// ranges, so one warpgroup reads both with the 16x32bx2 access shape
+// (threads 0-15 of a warp get A's rows, 16-31 B's rows).
+//   warp 0 / 2 : loader for slot 0 / 1 (lane 0 Q, lane 1 K, lane 2 V; TMA)
+//   warp 1 / 3 : MMA issuer for slot 0 / 1 (one thread)
+//   warps 4-7  : softmax + epilogue warpgroup of slot 0
+//   warps 8-11 : softmax + epilogue warpgroup of slot 1
+// Every wait on an mbarrier is bounded (2 s); on expiry the kernel records
+// a timeout in the status word, the other roles stop at their next wait,
+// in-flight copies and MMAs are drained (bounded), TMEM is freed and the
+// kernel returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "bsa_internal.cuh"
 
 namespace bsa {
-cudaError_t launch_attend_tc(const Problem &, const void *, const void *, const void *, const float *,
-                             const float *, const int32_t *, void *, uint32_t *, cudaStream_t) {
-    return cudaErrorNotSupported;
+namespace {
+
+constexpr int BK = 64;                      // tokens per block
+constexpr int HD = 64;                      // head dim
+constexpr int TILE = BK * HD * 2;           // bytes of one 64x64 bf16 tile
+constexpr int NSLOT = 2;
+constexpr int NTHREADS = 384;
+constexpr uint32_t TMEM_COLS = 512;         // per slot: S_A, S_B, O_A, O_B (64 columns each)
+constexpr float kRescaleLog2 = 8.0f;        // lazy rescale threshold (factor 256)
+constexpr unsigned long long kWaitNs = 2000000000ull;
+constexpr unsigned long long kDrainNs = 200000000ull;
+
+struct alignas(1024) SlotTiles {
+    uint8_t q[2][2][TILE];   // [buffer][A/B]
+    uint8_t k[2][2][TILE];   // [stage][A/B]
+    uint8_t v[2][2][TILE];   // [stage][A/B]
+    uint8_t p[2][TILE];      // [A/B]
+};
+static_assert(sizeof(SlotTiles) == 14 * TILE, "tile layout");
+
+struct SlotBars {
+    uint64_t q_full[2], q_empty[2];
+    uint64_t k_full[2], k_empty[2];
+    uint64_t v_full[2], v_empty[2];
+    uint64_t s_full, s_free, p_full, o_done, drain;
+};
+
+struct SharedStorage {
+    SlotTiles tiles[NSLOT];
+    SlotBars bars[NSLOT];
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+struct TcParams {
+    const int32_t *idx;     // [slabs*m][n]
+    const float *gates;     // [slabs*N][3]
+    const float *o_cg;      // [slabs*m][64]
+    __nv_bfloat16 *out;     // [slabs*N][64]
+    uint32_t *status;       // nullable
+    int64_t n_tokens;
+    int64_t total_pairs;
+    int m, n, w, pairs_per_slab;
+    float scale_log2;
+};
+
+// ---------------------------------------------------------------- PTX glue
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
 }
+__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for the phase of parity `parity`. Returns false if the CTA is
+// aborting or the wait expired (which starts the abort and flags a timeout).
+__device__ __noinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile int *abort_flag,
+                                      uint32_t *status) {
+    if (mbar_try_wait(b, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(b, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_ns() - t0 > kWaitNs) {
+                *abort_flag = 1;
+                if (status) atomicOr(status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+// Drain wait used on the abort path only: bounded, ignores the abort flag.
+__device__ __noinline__ void drain_bar(uint64_t *b, uint32_t parity) {
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(b, parity))
+        if (global_ns() - t0 > kDrainNs) return;
+}
+
+__device__ __forceinline__ void tma_load_tile(void *dst, const CUtensorMap *map, uint64_t *bar, int row) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(row)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 16 lanes x 16 columns twice: thread t of the warp gets TMEM lane (base + t%16),
+// columns [col, col+16) for t < 16 and [col+64, col+80) for t >= 16.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *r) {
+    uint32_t *u = reinterpret_cast<uint32_t *>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 64;"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *r) {
+    const uint32_t *u = reinterpret_cast<const uint32_t *>(r);
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 64, "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "r"(u[8]),
+        "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 descriptor version.
+__device__ __forceinline__ uint64_t smem_desc(const void *tile, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    const uint32_t a = smem_u32(tile);
+    uint64_t d = (uint64_t)((a >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+// K-major operand (rows of 64 bf16 = 128 B, 8-row groups 1024 B apart)
+__device__ __forceinline__ uint64_t desc_kmajor(const void *tile) { return smem_desc(tile, 16, 1024); }
+// MN-major operand (V as [key][d]: N = d contiguous, K = key rows 128 B apart)
+__device__ __forceinline__ uint64_t desc_mnmajor(const void *tile) { return smem_desc(tile, TILE, 1024); }
+
+// instruction descriptor: D f32, A/B bf16, M=64, N=64, A K-major, B K- or MN-major
+constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(64 >> 3) << 17) |
+                                ((uint32_t)(64 >> 4) << 24);
+constexpr uint32_t kIdescS = kIdescBase;
+constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);
+
+// ------------------------------------------------------------ work layout
+
+struct Pair {
+    int64_t slab;
+    int iA, iB;
+    bool validB;
+};
+__device__ __forceinline__ Pair pair_of(const TcParams &p, int64_t pr) {
+    Pair r;
+    r.slab = pr / p.pairs_per_slab;
+    r.iA = (int)(pr - r.slab * p.pairs_per_slab) * 2;
+    r.validB = r.iA + 1 < p.m;
+    r.iB = r.validB ? r.iA + 1 : r.iA;
+    return r;
+}
+// Key block of query block i at step t: local window first (t < L), then the
+// selected blocks. Out-of-range blocks are masked (loaded as block i, P = 0).
+__device__ __forceinline__ int step_block(const TcParams &p, int64_t slab, int i, int t, int L, bool &valid) {
+    int j;
+    if (t < L) {
+        j = i - p.w + t;
+    } else {
+        j = __ldg(p.idx + (slab * p.m + i) * (int64_t)p.n + (t - L));
+    }
+    valid = j >= 0 && j < p.m;
+    return valid ? j : i;
+}
+
+// ------------------------------------------------------------------ roles
+
+__device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUtensorMap *tk,
+                            const CUtensorMap *tv, SlotTiles &S, SlotBars &B, int slot, int lane,
+                            volatile int *abort_flag) {
+    if (lane > 2) return;
+    const int L = 2 * p.w + 1, T = L + p.n;
+    const int64_t first = 2 * (int64_t)blockIdx.x + slot, stride = 2 * (int64_t)gridDim.x;
+    uint32_t c = 0, g = 0;                 // pairs / steps issued by this lane
+    uint64_t *last_bar[2] = {nullptr, nullptr};
+    uint32_t last_par[2] = {0, 0};
+    bool ok = true;
+    for (int64_t pr = first; pr < p.total_pairs && ok; pr += stride, ++c) {
+        const Pair P = pair_of(p, pr);
+        const int64_t base = P.slab * p.n_tokens;
+        if (lane == 0) {                   // Q tiles of the pair (double buffered)
+            const int qb = c & 1;
+            if (!(ok = wait_bar(&B.q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+            mbar_expect_tx(&B.q_full[qb], 2 * TILE);
+            tma_load_tile(S.q[qb][0], tq, &B.q_full[qb], (int)(base + (int64_t)P.iA * BK));
+            tma_load_tile(S.q[qb][1], tq, &B.q_full[qb], (int)(base + (int64_t)P.iB * BK));
+            last_bar[c & 1] = &B.q_full[qb];
+            last_par[c & 1] = (c >> 1) & 1;
+            continue;
+        }
+        for (int t = 0; t < T; ++t, ++g) { // K (lane 1) or V (lane 2) tiles of every step
+            bool va, vb;
+            const int ja = step_block(p, P.slab, P.iA, t, L, va);
+            const int jb = step_block(p, P.slab, P.iB, t, L, vb);
+            if (lane == 1 && t >= L && (!va || !vb) && p.status) atomicOr(p.status, kStatusBadIndex);
+            const int st = g & 1;
+            uint64_t *full = lane == 1 ? &B.k_full[st] : &B.v_full[st];
+            uint64_t *empty = lane == 1 ? &B.k_empty[st] : &B.v_empty[st];
+            uint8_t(*dst)[TILE] = lane == 1 ? S.k[st] : S.v[st];
+            const CUtensorMap *map = lane == 1 ? tk : tv;
+            if (!(ok = wait_bar(empty, ((g >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+            mbar_expect_tx(full, 2 * TILE);
+            tma_load_tile(dst[0], map, full, (int)(base + (int64_t)ja * BK));
+            tma_load_tile(dst[1], map, full, (int)(base + (int64_t)jb * BK));
+            last_bar[g & 1] = full;
+            last_par[g & 1] = (g >> 1) & 1;
+        }
+    }
+    if (!ok) {                             // let copies in flight land before the CTA exits
+        for (int s = 0; s < 2; ++s)
+            if (last_bar[s]) drain_bar(last_bar[s], last_par[s]);
+    }
+}
+
+__device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t tmem_slot, int slot, int lane,
+                         volatile int *abort_flag) {
+    if (lane != 0) return;
+    const int L = 2 * p.w + 1, T = L + p.n;
+    const int64_t stride = 2 * (int64_t)gridDim.x;
+    const uint32_t tS = tmem_slot, tO = tmem_slot + 128;
+    uint32_t c = 0, g = 0;
+    bool ok = true;
+    for (int64_t pr = 2 * (int64_t)blockIdx.x + slot; pr < p.total_pairs && ok; pr += stride, ++c) {
+        const int qb = c & 1;
+        if (!(ok = wait_bar(&B.q_full[qb], (c >> 1) & 1, abort_flag, p.status))) break;
+        // S(gs) = Q·K(gs)ᵀ for both query blocks; needs K loaded and the previous S read out
+        auto issue_s = [&](uint32_t gs) -> bool {
+            const int ks = gs & 1;
+            if (!wait_bar(&B.k_full[ks], (gs >> 1) & 1, abort_flag, p.status)) return false;
+            if (gs > 0 && !wait_bar(&B.s_free, (gs - 1) & 1, abort_flag, p.status)) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint64_t a = desc_kmajor(S.q[qb][h]);
+                const uint64_t b = desc_kmajor(S.k[ks][h]);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) tc_mma(tS + h * 64, a + 2 * kk, b + 2 * kk, kIdescS, kk > 0);
+            }
+            tc_commit(&B.s_full);
+            tc_commit(&B.k_empty[ks]);
+            return true;
+        };
+        if (!(ok = issue_s(g))) break;
+        if (T == 1) tc_commit(&B.q_empty[qb]);
+        for (int t = 0; t < T; ++t, ++g) {
+            if (t + 1 < T) {                       // the next S runs while this step's softmax does
+                if (!(ok = issue_s(g + 1))) break;
+                if (t + 2 == T) tc_commit(&B.q_empty[qb]);
+            }
+            const int vs = g & 1;
+            if (!(ok = wait_bar(&B.p_full, g & 1, abort_flag, p.status))) break;
+            if (!(ok = wait_bar(&B.v_full[vs], (g >> 1) & 1, abort_flag, p.status))) break;
+            tc_fence_after();
+            const uint32_t accum = (t == 0 || t == L) ? 0u : 1u;   // each branch starts a fresh O
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint64_t a = desc_kmajor(S.p[h]);
+                const uint64_t b = desc_mnmajor(S.v[vs][h]);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc_mma(tO + h * 64, a + 2 * kk, b + 128 * kk, kIdescPV, accum | (kk > 0 ? 1u : 0u));
+            }
+            tc_commit(&B.o_done);
+            tc_commit(&B.v_empty[vs]);
+        }
+    }
+    // every MMA this thread issued must be complete before TMEM is freed
+    tc_commit(&B.drain);
+    drain_bar(&B.drain, 0);
+}
+
+__device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t tmem_slot, int slot,
+                             int wq, int lane, volatile int *abort_flag) {
+    const unsigned FULL = 0xffffffffu;
+    const int L = 2 * p.w + 1, T = L + p.n;
+    const int half = lane >> 4;            // 0: query block A, 1: query block B
+    const int r = 16 * wq + (lane & 15);   // row within the query block
+    const uint32_t tlane = (uint32_t)(32 * wq) << 16;
+    const uint32_t tS = tmem_slot + tlane, tO = tmem_slot + 128 + tlane;
+    uint8_t *prow = S.p[half] + (r >> 3) * 1024 + (r & 7) * 128;
+    const int sw = r & 7;
+    const float sl2 = p.scale_log2;
+    const int64_t stride = 2 * (int64_t)gridDim.x;
+    uint32_t g = 0;
+    bool ok = true;
+    auto wait_all = [&](uint64_t *b, uint32_t par) -> bool {
+        const bool mine = wait_bar(b, par, abort_flag, p.status);
+        return __all_sync(FULL, mine);
+    };
+    for (int64_t pr = 2 * (int64_t)blockIdx.x + slot; pr < p.total_pairs && ok; pr += stride) {
+        const Pair P = pair_of(p, pr);
+        const int i = half ? P.iB : P.iA;
+        const bool row_valid = half ? P.validB : true;
+        const int64_t tok = P.slab * p.n_tokens + (int64_t)i * BK + r;
+        const float *gp = p.gates + tok * 3;
+        const float g_cg = __ldg(gp), g_fg = __ldg(gp + 1), g_l = __ldg(gp + 2);
+        const float *ocg = p.o_cg + (P.slab * p.m + i) * (int64_t)HD;
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(ocg));
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(ocg + 32));
+        float acc[HD];
+#pragma unroll
+        for (int c = 0; c < HD; ++c) acc[c] = 0.f;
+        float m_used = -INFINITY, l_run = 0.f, l_local = 0.f;
+        for (int t = 0; t < T; ++t, ++g) {
+            bool valid;
+            (void)step_block(p, P.slab, i, t, L, valid);
+            valid = valid && row_valid;
+            if (t == L) {                      // the selection branch starts afresh
+                l_local = l_run;
+                l_run = 0.f;
+                m_used = -INFINITY;
+            }
+            // ---- scores of this step
+            if (!(ok = wait_all(&B.s_full, g & 1))) break;
+            tc_fence_after();
+            float s[64];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld16(tS + 16 * c, s + 16 * c);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&B.s_free);
+            // ---- softmax numerators against the (lazily updated) running max
+            float mx = -INFINITY;
+            if (valid) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
+                mx *= sl2;
+            }
+            const bool need = valid && m_used != -INFINITY && mx > m_used + kRescaleLog2;
+            const float m_old = m_used;
+            if (valid && (m_used == -INFINITY || need)) m_used = mx;
+            uint32_t pk[32];
+            float ls = 0.f;
+            if (valid) {
+                const float nm = -m_used;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float p0 = ex2(fmaf(s[2 * c], sl2, nm));
+                    const float p1 = ex2(fmaf(s[2 * c + 1], sl2, nm));
+                    pk[c] = pack_bf16(p0, p1);
+                    ls += bf16_lo(pk[c]) + bf16_hi(pk[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) pk[c] = 0u;
+            }
+            // ---- the previous P·V must be complete before P or O is touched
+            if (g > 0 && !(ok = wait_all(&B.o_done, (g - 1) & 1))) break;
+            tc_fence_after();
+            if (t == L) {
+                // close the local branch: acc = g_CG·o_CG + g_L·o_L
+                const float inv = l_local > 0.f ? g_l / l_local : 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float o[16];
+                    tmem_ld16(tO + 16 * c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) acc[16 * c + e] = fmaf(g_cg, __ldg(ocg + 16 * c + e), o[e] * inv);
+                }
+            } else if (__any_sync(FULL, need)) {
+                // rows whose running max grew by more than 2^8: rescale their O and sum
+                const float alpha = need ? ex2(m_old - m_used) : 1.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float o[16];
+                    tmem_ld16(tO + 16 * c, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) o[e] *= alpha;
+                    tmem_st16(tO + 16 * c, o);
+                }
+                tmem_wait_st();
+                l_run *= alpha;
+            }
+            l_run += ls;
+            // ---- P row -> shared memory (K-major, 128-byte swizzle)
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint4 v4 = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+                *reinterpret_cast<uint4 *>(prow + ((ch ^ sw) << 4)) = v4;
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&B.p_full);
+        }
+        if (!ok) break;
+        // ---- epilogue: out = acc + g_FG·o_FG
+        if (!(ok = wait_all(&B.o_done, (g - 1) & 1))) break;
+        tc_fence_after();
+        const float inv = l_run > 0.f ? g_fg / l_run : 0.f;
+        __nv_bfloat16 *dst = p.out + tok * HD;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            float o[16];
+            tmem_ld16(tO + 16 * c, o);
+            tmem_wait_ld();
+            uint32_t w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                w8[e] = pack_bf16(fmaf(o[2 * e], inv, acc[16 * c + 2 * e]),
+                                  fmaf(o[2 * e + 1], inv, acc[16 * c + 2 * e + 1]));
+            if (row_valid) {
+                uint4 *d4 = reinterpret_cast<uint4 *>(dst + 16 * c);
+                d4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+                d4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+            }
+        }
+        tc_fence_before();
+    }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                 const __grid_constant__ CUtensorMap tv, const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    SharedStorage &sh = *reinterpret_cast<SharedStorage *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int *abort_flag = &sh.abort_flag;
+
+    if (threadIdx.x == 0) {
+        sh.abort_flag = 0;
+        for (int s = 0; s < NSLOT; ++s) {
+            SlotBars &B = sh.bars[s];
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&B.q_full[b], 1);
+                mbar_init(&B.q_empty[b], 1);
+                mbar_init(&B.k_full[b], 1);
+                mbar_init(&B.k_empty[b], 1);
+                mbar_init(&B.v_full[b], 1);
+                mbar_init(&B.v_empty[b], 1);
+            }
+            mbar_init(&B.s_full, 1);
+            mbar_init(&B.s_free, 4);
+            mbar_init(&B.p_full, 4);
+            mbar_init(&B.o_done, 1);
+            mbar_init(&B.drain, 1);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&sh.tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+
+    if (warp < 4) {
+        const int slot = warp >> 1;
+        if ((warp & 1) == 0)
+            loader_role(p, &tq, &tk, &tv, sh.tiles[slot], sh.bars[slot], slot, lane, abort_flag);
+        else
+            mma_role(p, sh.tiles[slot], sh.bars[slot], tmem + 256u * slot, slot, lane, abort_flag);
+    } else {
+        const int slot = (warp - 4) >> 2;
+        softmax_role(p, sh.tiles[slot], sh.bars[slot], tmem + 256u * slot, slot, warp & 3, lane, abort_flag);
+    }
+    __syncwarp();                          // reconverge role lanes before the CTA barrier
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// --------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+bool make_tile_map(CUtensorMap *map, const void *base, uint64_t rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)HD, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)HD * 2};
+    cuuint32_t box[2] = {(cuuint32_t)HD, (cuuint32_t)BK};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+}  // namespace
+
+cudaError_t launch_attend_tc(const Problem &pb, const void *q, const void *k, const void *v,
+                             const float *gates, const float *o_cg, const int32_t *idx, void *out,
+                             uint32_t *status, cudaStream_t stream) {
+    if (pb.dtype != BSA_BF16 || pb.block_size != BK || pb.head_dim != HD) return cudaErrorNotSupported;
+    const int64_t rows = pb.slabs * pb.n_tokens;
+    if (rows > 0x7fffffffLL) return cudaErrorNotSupported;       // TMA row coordinate is int32
+    CUtensorMap tq, tk, tv;
+    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows))
+        return cudaErrorNotSupported;
+    TcParams p;
+    p.idx = idx;
+    p.gates = gates;
+    p.o_cg = o_cg;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.status = status;
+    p.n_tokens = pb.n_tokens;
+    p.m = (int)pb.m;
+    p.n = (int)pb.top_n;
+    p.w = (int)pb.window;
+    p.pairs_per_slab = (int)((pb.m + 1) / 2);
+    p.total_pairs = pb.slabs * p.pairs_per_slab;
+    p.scale_log2 = pb.scale * 1.4426950408889634f;
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorNotSupported;
+    const int64_t want = (p.total_pairs + NSLOT - 1) / NSLOT;
+    const int grid = (int)(want < sms ? want : sms);
+    const size_t smem = sizeof(SharedStorage) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attend_tc_kernel<<<grid, NTHREADS, smem, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
 }  // namespace bsa
