@@ -21,6 +21,7 @@ STATUS_NAMES = {
 }
 EXPORTS = ("bsa_pool", "bsa_compress_select", "bsa_fine_attention", "bsa_workspace_size",
            "bsa_forward", "bsa_check_status", "bsa_status_string", "bsa_forward_noalloc")
+TESTING_EXPORTS = ("bsa_testing_fine_attention_withhold",)
 
 
 class BsaConfig(ctypes.Structure):
@@ -56,6 +57,7 @@ def load() -> ctypes.CDLL:
         "bsa_check_status": [P, P],
         "bsa_status_string": [ctypes.c_int],
         "bsa_forward_noalloc": [C, P, P, P, P, P, P, P, P],
+        "bsa_testing_fine_attention_withhold": [C, P, P, P, P, P, P, P, P, ctypes.c_int64, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)

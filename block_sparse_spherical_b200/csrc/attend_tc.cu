@@ -79,6 +79,7 @@ struct TcParams {
     int64_t total_pairs;
     int m, n, w, pairs_per_slab;
     float scale_log2;
+    int64_t withhold_v_step;   // test hook, -1 = off
 };
 
 // ---------------------------------------------------------------- PTX glue
@@ -283,6 +284,7 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
             uint8_t(*dst)[TILE] = lane == 1 ? S.k[st] : S.v[st];
             const CUtensorMap *map = lane == 1 ? tk : tv;
             if (!(ok = wait_bar(empty, ((g >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+            if (lane == 2 && (int64_t)g == p.withhold_v_step && blockIdx.x == 0 && slot == 0) continue;
             mbar_expect_tx(full, 2 * TILE);
             tma_load_tile(dst[0], map, full, (int)(base + (int64_t)ja * BK));
             tma_load_tile(dst[1], map, full, (int)(base + (int64_t)jb * BK));
@@ -616,6 +618,7 @@ cudaError_t launch_attend_tc(const Problem &pb, const void *q, const void *k, co
     p.pairs_per_slab = (int)((pb.m + 1) / 2);
     p.total_pairs = pb.slabs * p.pairs_per_slab;
     p.scale_log2 = pb.scale * 1.4426950408889634f;
+    p.withhold_v_step = pb.withhold_v_step;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorNotSupported;
     const int64_t want = (p.total_pairs + NSLOT - 1) / NSLOT;

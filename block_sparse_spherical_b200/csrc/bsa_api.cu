@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include "bsa_internal.cuh"
+#include "bsa_testing.h"
 
 namespace {
 
@@ -267,4 +268,25 @@ extern "C" bsa_status bsa_forward_noalloc(const bsa_config *cfg, const void *q, 
     if (e == cudaSuccess) e = bsa::launch_compress_select(p, qbar, kbar, vbar, ocg, idx, stream);
     if (e == cudaSuccess) e = launch_fine(p, q, k, v, gates, ocg, idx, out, status_word, stream);
     return from_cuda(e);
+}
+
+// ---------------------------------------------------------------------------
+// Test hook (include/bsa_testing.h): the tensor-core fine-attention kernel
+// with one V copy withheld, so that a bounded wait expires on purpose.
+// ---------------------------------------------------------------------------
+extern "C" bsa_status bsa_testing_fine_attention_withhold(const bsa_config *cfg, const void *q, const void *k,
+                                                           const void *v, const float *gates,
+                                                           const float *o_cg_block, const int32_t *sel_idx,
+                                                           void *out, uint32_t *status_word,
+                                                           int64_t withhold_v_step, cudaStream_t stream) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (!q || !k || !v || !gates || !o_cg_block || !sel_idx || !out || !status_word) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gates) || !aligned16(o_cg_block) ||
+        !aligned16(sel_idx) || !aligned16(out) || ((uintptr_t)status_word & 3u))
+        return BSA_ERR_ALIGNMENT;
+    if (withhold_v_step < 0) return BSA_ERR_INVALID_ARG;
+    p.withhold_v_step = withhold_v_step;
+    return from_cuda(bsa::launch_attend_tc(p, q, k, v, gates, o_cg_block, sel_idx, out, status_word, stream));
 }

@@ -22,6 +22,9 @@ struct Problem {
     int64_t slabs;    // batch * heads
     bsa_dtype dtype;
     float scale;      // logit scale s
+    // Test hook: when >= 0 the tensor-core kernel's first pipeline skips the V
+    // copy of this step, so that the wait for it expires (bounded-wait test).
+    int64_t withhold_v_step = -1;
 };
 
 // Launchers (return cudaGetLastError()).

@@ -9,7 +9,7 @@ import pytest
 from block_sparse_spherical_b200 import abi, build
 from block_sparse_spherical_b200.configs import CONFIGS
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "bsa.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
 
 
 @pytest.fixture(scope="module")
@@ -18,14 +18,18 @@ def lib():
     return abi.load()
 
 
-def declared_functions():
-    src = open(HEADER).read()
-    return re.findall(r"BSA_API\s+[\w\s\*]+?\b(bsa_\w+)\s*\(", src)
+def declared_functions(header=None):
+    names = []
+    for h in sorted(os.listdir(INCLUDE)):
+        if h.endswith(".h") and (header is None or h == header):
+            src = open(os.path.join(INCLUDE, h)).read()
+            names += re.findall(r"BSA_API\s+[\w\s\*]+?\b(bsa_\w+)\s*\(", src)
+    return names
 
 
 def test_header_declares_the_binding_names():
-    names = declared_functions()
-    assert sorted(names) == sorted(abi.EXPORTS)
+    assert sorted(declared_functions("bsa.h")) == sorted(abi.EXPORTS)
+    assert sorted(declared_functions("bsa_testing.h")) == sorted(abi.TESTING_EXPORTS)
 
 
 def test_library_exports_every_declared_symbol(lib):
