@@ -13,16 +13,17 @@
 // selection branch reuses the same TMEM accumulator; the epilogue adds
 // g_FG·o_FG and stores bf16.
 //
-// Organisation: a persistent grid of one CTA per SM, 384 threads, two
+// Organisation: a persistent grid of one CTA per SM, 640 threads, two
 // independent pipelines ("slots") per CTA. A slot works on a pair of
 // neighbouring query blocks (A, B) at a time; their M=64 accumulators live
 // in TMEM lanes 0-15 of each 32-lane sub-partition at adjacent 64-column
-// ranges, so one warpgroup reads both with the 16x32bx2 access shape
-// (threads 0-15 of a warp get A's rows, 16-31 B's rows).
-//   warp 0 / 2 : loader for slot 0 / 1 (lane 0 Q, lane 1 K, lane 2 V; TMA)
-//   warp 1 / 3 : MMA issuer for slot 0 / 1 (one thread)
-//   warps 4-7  : softmax + epilogue warpgroup of slot 0
-//   warps 8-11 : softmax + epilogue warpgroup of slot 1
+// ranges. Each query block has its own softmax warpgroup; with the 16x32bx2
+// access shape a warp reads 16 rows, threads t and t+16 sharing a row
+// (columns 0-31 and 32-63).
+//   warp 0 / 2  : loader for slot 0 / 1 (lane 0 Q, lane 1 K, lane 2 V; TMA)
+//   warp 1 / 3  : MMA issuer for slot 0 / 1 (one thread)
+//   warps 4-11  : softmax + epilogue of slot 0 (4-7 block A, 8-11 block B)
+//   warps 12-19 : softmax + epilogue of slot 1
 // Every wait on an mbarrier is bounded (2 s); on expiry the kernel records
 // a timeout in the status word, the other roles stop at their next wait,
 // in-flight copies and MMAs are drained (bounded), TMEM is freed and the
@@ -41,7 +42,7 @@ constexpr int BK = 64;                      // tokens per block
 constexpr int HD = 64;                      // head dim
 constexpr int TILE = BK * HD * 2;           // bytes of one 64x64 bf16 tile
 constexpr int NSLOT = 2;
-constexpr int NTHREADS = 384;
+constexpr int NTHREADS = 640;
 constexpr uint32_t TMEM_COLS = 512;         // per slot: S_A, S_B, O_A, O_B (64 columns each)
 constexpr float kRescaleLog2 = 8.0f;        // lazy rescale threshold (factor 256)
 constexpr unsigned long long kWaitNs = 2000000000ull;
@@ -132,6 +133,10 @@ __device__ __noinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile int
         }
     }
 }
+__device__ __forceinline__ bool wait_fast(uint64_t *b, uint32_t parity, volatile int *abort_flag,
+                                          uint32_t *status) {
+    return mbar_try_wait(b, parity) || wait_bar(b, parity, abort_flag, status);
+}
 // Drain wait used on the abort path only: bounded, ignores the abort flag.
 __device__ __noinline__ void drain_bar(uint64_t *b, uint32_t parity) {
     const uint64_t t0 = global_ns();
@@ -164,12 +169,12 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
 }
 
 // 16 lanes x 16 columns twice: thread t of the warp gets TMEM lane (base + t%16),
-// columns [col, col+16) for t < 16 and [col+64, col+80) for t >= 16.
+// columns [col, col+16) for t < 16 and [col+32, col+48) for t >= 16.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *r) {
     uint32_t *u = reinterpret_cast<uint32_t *>(r);
     asm volatile(
         "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 64;"
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 32;"
         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
           "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
         : "r"(taddr));
@@ -177,7 +182,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *r) {
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *r) {
     const uint32_t *u = reinterpret_cast<const uint32_t *>(r);
     asm volatile(
-        "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 64, "
+        "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 32, "
         "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
         "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "r"(u[8]),
         "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
@@ -196,8 +201,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
-__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 descriptor version.
 __device__ __forceinline__ uint64_t smem_desc(const void *tile, uint32_t lbo_bytes, uint32_t sbo_bytes) {
@@ -235,14 +238,14 @@ __device__ __forceinline__ Pair pair_of(const TcParams &p, int64_t pr) {
     r.iB = r.validB ? r.iA + 1 : r.iA;
     return r;
 }
-// Key block of query block i at step t: local window first (t < L), then the
-// selected blocks. Out-of-range blocks are masked (loaded as block i, P = 0).
-__device__ __forceinline__ int step_block(const TcParams &p, int64_t slab, int i, int t, int L, bool &valid) {
+// Key block of query block i at step t: the n selected blocks first (t < n),
+// then the local window. Out-of-range blocks are masked (loaded as block i, P = 0).
+__device__ __forceinline__ int step_block(const TcParams &p, int64_t slab, int i, int t, bool &valid) {
     int j;
-    if (t < L) {
-        j = i - p.w + t;
+    if (t < p.n) {
+        j = __ldg(p.idx + (slab * p.m + i) * (int64_t)p.n + t);
     } else {
-        j = __ldg(p.idx + (slab * p.m + i) * (int64_t)p.n + (t - L));
+        j = i - p.w + (t - p.n);
     }
     valid = j >= 0 && j < p.m;
     return valid ? j : i;
@@ -275,9 +278,9 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
         }
         for (int t = 0; t < T; ++t, ++g) { // K (lane 1) or V (lane 2) tiles of every step
             bool va, vb;
-            const int ja = step_block(p, P.slab, P.iA, t, L, va);
-            const int jb = step_block(p, P.slab, P.iB, t, L, vb);
-            if (lane == 1 && t >= L && (!va || !vb) && p.status) atomicOr(p.status, kStatusBadIndex);
+            const int ja = step_block(p, P.slab, P.iA, t, va);
+            const int jb = step_block(p, P.slab, P.iB, t, vb);
+            if (lane == 1 && t < p.n && (!va || !vb) && p.status) atomicOr(p.status, kStatusBadIndex);
             const int st = g & 1;
             uint64_t *full = lane == 1 ? &B.k_full[st] : &B.v_full[st];
             uint64_t *empty = lane == 1 ? &B.k_empty[st] : &B.v_empty[st];
@@ -312,8 +315,8 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
         // S(gs) = Q·K(gs)ᵀ for both query blocks; needs K loaded and the previous S read out
         auto issue_s = [&](uint32_t gs) -> bool {
             const int ks = gs & 1;
-            if (!wait_bar(&B.k_full[ks], (gs >> 1) & 1, abort_flag, p.status)) return false;
-            if (gs > 0 && !wait_bar(&B.s_free, (gs - 1) & 1, abort_flag, p.status)) return false;
+            if (!wait_fast(&B.k_full[ks], (gs >> 1) & 1, abort_flag, p.status)) return false;
+            if (gs > 0 && !wait_fast(&B.s_free, (gs - 1) & 1, abort_flag, p.status)) return false;
             tc_fence_after();
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -334,10 +337,10 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
                 if (t + 2 == T) tc_commit(&B.q_empty[qb]);
             }
             const int vs = g & 1;
-            if (!(ok = wait_bar(&B.p_full, g & 1, abort_flag, p.status))) break;
-            if (!(ok = wait_bar(&B.v_full[vs], (g >> 1) & 1, abort_flag, p.status))) break;
+            if (!(ok = wait_fast(&B.p_full, g & 1, abort_flag, p.status))) break;
+            if (!(ok = wait_fast(&B.v_full[vs], (g >> 1) & 1, abort_flag, p.status))) break;
             tc_fence_after();
-            const uint32_t accum = (t == 0 || t == L) ? 0u : 1u;   // each branch starts a fresh O
+            const uint32_t accum = (t == 0 || t == p.n) ? 0u : 1u;   // each branch starts a fresh O
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const uint64_t a = desc_kmajor(S.p[h]);
@@ -355,14 +358,16 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
     drain_bar(&B.drain, 0);
 }
 
+// One warpgroup per query block of the pair. Thread (wq, lane): row
+// r = 16*wq + lane%16, columns 32*(lane/16) .. +31 of the block's S and O.
 __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t tmem_slot, int slot,
-                             int wq, int lane, volatile int *abort_flag) {
+                             int half, int wq, int lane, volatile int *abort_flag) {
     const unsigned FULL = 0xffffffffu;
     const int L = 2 * p.w + 1, T = L + p.n;
-    const int half = lane >> 4;            // 0: query block A, 1: query block B
+    const int ch = lane >> 4;              // column half of the row
     const int r = 16 * wq + (lane & 15);   // row within the query block
     const uint32_t tlane = (uint32_t)(32 * wq) << 16;
-    const uint32_t tS = tmem_slot + tlane, tO = tmem_slot + 128 + tlane;
+    const uint32_t tS = tmem_slot + 64 * half + tlane, tO = tmem_slot + 128 + 64 * half + tlane;
     uint8_t *prow = S.p[half] + (r >> 3) * 1024 + (r & 7) * 128;
     const int sw = r & 7;
     const float sl2 = p.scale_log2;
@@ -370,7 +375,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
     uint32_t g = 0;
     bool ok = true;
     auto wait_all = [&](uint64_t *b, uint32_t par) -> bool {
-        const bool mine = wait_bar(b, par, abort_flag, p.status);
+        const bool mine = wait_fast(b, par, abort_flag, p.status);
         return __all_sync(FULL, mine);
     };
     for (int64_t pr = 2 * (int64_t)blockIdx.x + slot; pr < p.total_pairs && ok; pr += stride) {
@@ -380,28 +385,40 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
         const int64_t tok = P.slab * p.n_tokens + (int64_t)i * BK + r;
         const float *gp = p.gates + tok * 3;
         const float g_cg = __ldg(gp), g_fg = __ldg(gp + 1), g_l = __ldg(gp + 2);
-        const float *ocg = p.o_cg + (P.slab * p.m + i) * (int64_t)HD;
+        const float *ocg = p.o_cg + (P.slab * p.m + i) * (int64_t)HD + 32 * ch;
         asm volatile("prefetch.global.L1 [%0];" ::"l"(ocg));
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(ocg + 32));
-        float acc[HD];
-#pragma unroll
-        for (int c = 0; c < HD; ++c) acc[c] = 0.f;
-        float m_used = -INFINITY, l_run = 0.f, l_local = 0.f;
+        // validity of the n selected blocks of this query block, as a bit mask
+        uint64_t selmask;
+        {
+            const int32_t *ix = p.idx + (P.slab * p.m + i) * (int64_t)p.n;
+            const int j0 = lane < p.n ? __ldg(ix + lane) : 0;
+            const int j1 = lane + 32 < p.n ? __ldg(ix + lane + 32) : 0;
+            const unsigned lo = __ballot_sync(FULL, j0 >= 0 && j0 < p.m);
+            const unsigned hi = __ballot_sync(FULL, j1 >= 0 && j1 < p.m);
+            selmask = ((uint64_t)hi << 32) | lo;
+        }
+        float acc[32];
+        float m_used = -INFINITY, l_run = 0.f, l_sel = 0.f;
         for (int t = 0; t < T; ++t, ++g) {
             bool valid;
-            (void)step_block(p, P.slab, i, t, L, valid);
+            if (t < p.n) {
+                valid = (selmask >> t) & 1u;
+            } else {
+                const int j = i - p.w + (t - p.n);
+                valid = j >= 0 && j < p.m;
+            }
             valid = valid && row_valid;
-            if (t == L) {                      // the selection branch starts afresh
-                l_local = l_run;
+            if (t == p.n) {                    // the local branch starts afresh
+                l_sel = l_run;
                 l_run = 0.f;
                 m_used = -INFINITY;
             }
             // ---- scores of this step
             if (!(ok = wait_all(&B.s_full, g & 1))) break;
             tc_fence_after();
-            float s[64];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld16(tS + 16 * c, s + 16 * c);
+            float s[32];
+            tmem_ld16(tS, s);
+            tmem_ld16(tS + 16, s + 16);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -410,35 +427,36 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             float mx = -INFINITY;
             if (valid) {
 #pragma unroll
-                for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
-                mx *= sl2;
+                for (int c = 0; c < 32; ++c) mx = fmaxf(mx, s[c]);
             }
+            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16)) * sl2;
             const bool need = valid && m_used != -INFINITY && mx > m_used + kRescaleLog2;
             const float m_old = m_used;
             if (valid && (m_used == -INFINITY || need)) m_used = mx;
-            uint32_t pk[32];
+            uint32_t pk[16];
             float ls = 0.f;
             if (valid) {
                 const float nm = -m_used;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
+                for (int c = 0; c < 16; ++c) {
                     const float p0 = ex2(fmaf(s[2 * c], sl2, nm));
                     const float p1 = ex2(fmaf(s[2 * c + 1], sl2, nm));
                     pk[c] = pack_bf16(p0, p1);
-                    ls += bf16_lo(pk[c]) + bf16_hi(pk[c]);
+                    ls += p0 + p1;
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) pk[c] = 0u;
+                for (int c = 0; c < 16; ++c) pk[c] = 0u;
             }
             // ---- the previous P·V must be complete before P or O is touched
             if (g > 0 && !(ok = wait_all(&B.o_done, (g - 1) & 1))) break;
             tc_fence_after();
-            if (t == L) {
-                // close the local branch: acc = g_CG·o_CG + g_L·o_L
-                const float inv = l_local > 0.f ? g_l / l_local : 0.f;
+            if (t == p.n) {
+                // close the selection branch: acc = g_CG·o_CG + g_FG·o_FG
+                const float l = l_sel + __shfl_xor_sync(FULL, l_sel, 16);
+                const float inv = l > 0.f ? g_fg / l : 0.f;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 2; ++c) {
                     float o[16];
                     tmem_ld16(tO + 16 * c, o);
                     tmem_wait_ld();
@@ -449,7 +467,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 // rows whose running max grew by more than 2^8: rescale their O and sum
                 const float alpha = need ? ex2(m_old - m_used) : 1.f;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < 2; ++c) {
                     float o[16];
                     tmem_ld16(tO + 16 * c, o);
                     tmem_wait_ld();
@@ -461,11 +479,12 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 l_run *= alpha;
             }
             l_run += ls;
-            // ---- P row -> shared memory (K-major, 128-byte swizzle)
+            // ---- P (this thread's 32 columns of the row) -> shared memory, K-major 128-byte swizzle
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const uint4 v4 = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-                *reinterpret_cast<uint4 *>(prow + ((ch ^ sw) << 4)) = v4;
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const int chunk = 4 * ch + c4;
+                const uint4 v4 = make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
+                *reinterpret_cast<uint4 *>(prow + ((chunk ^ sw) << 4)) = v4;
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
@@ -473,25 +492,24 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             if (lane == 0) mbar_arrive(&B.p_full);
         }
         if (!ok) break;
-        // ---- epilogue: out = acc + g_FG·o_FG
+        // ---- epilogue: out = acc + g_L·o_L
         if (!(ok = wait_all(&B.o_done, (g - 1) & 1))) break;
         tc_fence_after();
-        const float inv = l_run > 0.f ? g_fg / l_run : 0.f;
-        __nv_bfloat16 *dst = p.out + tok * HD;
+        const float l = l_run + __shfl_xor_sync(FULL, l_run, 16);
+        const float inv = l > 0.f ? g_l / l : 0.f;
+        uint4 *d4 = reinterpret_cast<uint4 *>(p.out + tok * HD + 32 * ch);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
             float o[16];
             tmem_ld16(tO + 16 * c, o);
             tmem_wait_ld();
             uint32_t w8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                w8[e] = pack_bf16(fmaf(o[2 * e], inv, acc[16 * c + 2 * e]),
-                                  fmaf(o[2 * e + 1], inv, acc[16 * c + 2 * e + 1]));
+                w8[e] = pack_bf16(fmaf(o[2 * e], inv, acc[16 * c + 2 * e]), fmaf(o[2 * e + 1], inv, acc[16 * c + 2 * e + 1]));
             if (row_valid) {
-                uint4 *d4 = reinterpret_cast<uint4 *>(dst + 16 * c);
-                d4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-                d4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+                d4[2 * c] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+                d4[2 * c + 1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
             }
         }
         tc_fence_before();
@@ -520,8 +538,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
                 mbar_init(&B.v_empty[b], 1);
             }
             mbar_init(&B.s_full, 1);
-            mbar_init(&B.s_free, 4);
-            mbar_init(&B.p_full, 4);
+            mbar_init(&B.s_free, 8);
+            mbar_init(&B.p_full, 8);
             mbar_init(&B.o_done, 1);
             mbar_init(&B.drain, 1);
         }
@@ -546,8 +564,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
         else
             mma_role(p, sh.tiles[slot], sh.bars[slot], tmem + 256u * slot, slot, lane, abort_flag);
     } else {
-        const int slot = (warp - 4) >> 2;
-        softmax_role(p, sh.tiles[slot], sh.bars[slot], tmem + 256u * slot, slot, warp & 3, lane, abort_flag);
+        const int slot = (warp - 4) >> 3;
+        const int half = ((warp - 4) >> 2) & 1;
+        softmax_role(p, sh.tiles[slot], sh.bars[slot], tmem + 256u * slot, slot, half, warp & 3, lane,
+                     abort_flag);
     }
     __syncwarp();                          // reconverge role lanes before the CTA barrier
 
