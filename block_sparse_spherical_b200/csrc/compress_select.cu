@@ -15,6 +15,9 @@
 // tx+16jj (jj<4) and its output columns are tx*(D/16)..+D/16. A row is thus
 // owned by the 16 lanes of one half-warp, which also hold that row's sorted
 // top-n list (entry e = tx + 16*slot) and update it with shuffles only.
+// Both products use the packed two-lane fp32 FMA of sm_100 (__ffma2_rn):
+// the logits pair partial sums over even/odd feature indices, P·v̄ pairs two
+// rows of P (stored transposed in shared memory) against a duplicated v̄.
 #include <math_constants.h>
 
 #include "bsa_internal.cuh"
@@ -81,7 +84,7 @@ compress_select_kernel(const float *__restrict__ qbar, const float *__restrict__
     load_rows<D>(Vs, v, 0, m, tid);
     cp_async_commit();
 
-    float o[4][DPT];
+    float2 op[2][DPT];   // (row 4ty+2k, row 4ty+2k+1) for output column c
     float mrun[4], lrun[4];
     float lv[4][NPL];
     int li[4][NPL];
@@ -89,8 +92,9 @@ compress_select_kernel(const float *__restrict__ qbar, const float *__restrict__
     for (int i = 0; i < 4; ++i) {
         mrun[i] = -CUDART_INF_F;
         lrun[i] = 0.f;
+        if (i < 2)
 #pragma unroll
-        for (int c = 0; c < DPT; ++c) o[i][c] = 0.f;
+            for (int c = 0; c < DPT; ++c) op[i][c] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int h = 0; h < NPL; ++h) { lv[i][h] = -CUDART_INF_F; li[i][h] = 0x7fffffff; }
     }
@@ -114,33 +118,34 @@ compress_select_kernel(const float *__restrict__ qbar, const float *__restrict__
 
         // ---- logits of the tile: s[i][jj] for row 4ty+i, key col0+tx+16jj
         float s[4][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) s[i][jj] = 0.f;
-#pragma unroll 4
-        for (int c = 0; c < D; c += 4) {
-            float4 qa[4], kb[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) qa[i] = *reinterpret_cast<const float4 *>(Qs + (4 * ty + i) * LDS + c);
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) kb[jj] = *reinterpret_cast<const float4 *>(Kt + (tx + 16 * jj) * LDS + c);
+        {
+            float2 sp[4][4];   // (even-feature, odd-feature) partial sums
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    s[i][jj] = fmaf(qa[i].x, kb[jj].x, s[i][jj]);
-                    s[i][jj] = fmaf(qa[i].y, kb[jj].y, s[i][jj]);
-                    s[i][jj] = fmaf(qa[i].z, kb[jj].z, s[i][jj]);
-                    s[i][jj] = fmaf(qa[i].w, kb[jj].w, s[i][jj]);
-                }
-        }
-        // log2-domain logits; columns past m do not exist
+                for (int jj = 0; jj < 4; ++jj) sp[i][jj] = make_float2(0.f, 0.f);
+#pragma unroll 1
+            for (int c = 0; c < D; c += 4) {
+                float4 qa[4], kb[4];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const bool ok = col0 + tx + 16 * jj < m;
+                for (int i = 0; i < 4; ++i) qa[i] = *reinterpret_cast<const float4 *>(Qs + (4 * ty + i) * LDS + c);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) s[i][jj] = ok ? s[i][jj] * scale_log2 : -CUDART_INF_F;
+                for (int jj = 0; jj < 4; ++jj) kb[jj] = *reinterpret_cast<const float4 *>(Kt + (tx + 16 * jj) * LDS + c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        sp[i][jj] = __ffma2_rn(make_float2(qa[i].x, qa[i].y), make_float2(kb[jj].x, kb[jj].y), sp[i][jj]);
+                        sp[i][jj] = __ffma2_rn(make_float2(qa[i].z, qa[i].w), make_float2(kb[jj].z, kb[jj].w), sp[i][jj]);
+                    }
+            }
+            // log2-domain logits; columns past m do not exist
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const bool ok = col0 + tx + 16 * jj < m;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s[i][jj] = ok ? (sp[i][jj].x + sp[i][jj].y) * scale_log2 : -CUDART_INF_F;
+            }
         }
 
         // ---- top-n merge (rows of this half-warp), candidates in any order
@@ -224,36 +229,39 @@ compress_select_kernel(const float *__restrict__ qbar, const float *__restrict__
             for (int jj = 0; jj < 4; ++jj) {
                 const float pexp = exp2f(s[i][jj] - mnew);
                 ls += pexp;
-                Ps[(4 * ty + i) * LDS + tx + 16 * jj] = pexp;
+                s[i][jj] = pexp;
             }
             lrun[i] = lrun[i] * alpha + ls;
 #pragma unroll
-            for (int c = 0; c < DPT; ++c) o[i][c] *= alpha;
+            for (int c = 0; c < DPT; ++c) {
+                if (i & 1) op[i >> 1][c].y *= alpha;
+                else op[i >> 1][c].x *= alpha;
+            }
         }
+        // P transposed: Ps[key][row], the thread's 4 rows as one 16-byte store per key
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+            *reinterpret_cast<float4 *>(Ps + (tx + 16 * jj) * LDS + 4 * ty) = make_float4(s[0][jj], s[1][jj], s[2][jj], s[3][jj]);
         __syncthreads();
 
-        // ---- o += P · v̄_tile
+        // ---- o += P · v̄_tile (rows paired: (o[0], o[1]) and (o[2], o[3]) per column)
 #pragma unroll 4
-        for (int j = 0; j < BN; j += 4) {
-            float4 pa[4];
+        for (int j = 0; j < BN; ++j) {
+            const float4 pr = *reinterpret_cast<const float4 *>(Ps + j * LDS + 4 * ty);
+            float vv[DPT];
+            if constexpr (DPT == 4) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(Vt + j * LDS + tx * 4);
+                vv[0] = t4.x; vv[1] = t4.y; vv[2] = t4.z; vv[3] = t4.w;
+            } else {
+                const float2 t2 = *reinterpret_cast<const float2 *>(Vt + j * LDS + tx * 2);
+                vv[0] = t2.x; vv[1] = t2.y;
+            }
+            const float2 p01 = make_float2(pr.x, pr.y), p23 = make_float2(pr.z, pr.w);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) pa[i] = *reinterpret_cast<const float4 *>(Ps + (4 * ty + i) * LDS + j);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float vv[DPT];
-                if constexpr (DPT == 4) {
-                    const float4 t4 = *reinterpret_cast<const float4 *>(Vt + (j + u) * LDS + tx * 4);
-                    vv[0] = t4.x; vv[1] = t4.y; vv[2] = t4.z; vv[3] = t4.w;
-                } else {
-                    const float2 t2 = *reinterpret_cast<const float2 *>(Vt + (j + u) * LDS + tx * 2);
-                    vv[0] = t2.x; vv[1] = t2.y;
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float pu = u == 0 ? pa[i].x : u == 1 ? pa[i].y : u == 2 ? pa[i].z : pa[i].w;
-#pragma unroll
-                    for (int c = 0; c < DPT; ++c) o[i][c] = fmaf(pu, vv[c], o[i][c]);
-                }
+            for (int c = 0; c < DPT; ++c) {
+                const float2 v2 = make_float2(vv[c], vv[c]);
+                op[0][c] = __ffma2_rn(p01, v2, op[0][c]);
+                op[1][c] = __ffma2_rn(p23, v2, op[1][c]);
             }
         }
         __syncthreads();   // Ps and this K/V buffer are rewritten next
@@ -268,11 +276,14 @@ compress_select_kernel(const float *__restrict__ qbar, const float *__restrict__
         const int r = row0 + 4 * ty + i;
         if (r < m) {
             const float inv = 1.0f / l;
+            float oi[DPT];
+#pragma unroll
+            for (int c = 0; c < DPT; ++c) oi[c] = ((i & 1) ? op[i >> 1][c].y : op[i >> 1][c].x) * inv;
             float *dst = o_cg + (slab * m + r) * (int64_t)D + tx * DPT;
             if constexpr (DPT == 4)
-                *reinterpret_cast<float4 *>(dst) = make_float4(o[i][0] * inv, o[i][1] * inv, o[i][2] * inv, o[i][3] * inv);
+                *reinterpret_cast<float4 *>(dst) = make_float4(oi[0], oi[1], oi[2], oi[3]);
             else
-                *reinterpret_cast<float2 *>(dst) = make_float2(o[i][0] * inv, o[i][1] * inv);
+                *reinterpret_cast<float2 *>(dst) = make_float2(oi[0], oi[1]);
             int32_t *ix = idx_out + (slab * m + r) * (int64_t)n;
 #pragma unroll
             for (int h = 0; h < NPL; ++h) {
