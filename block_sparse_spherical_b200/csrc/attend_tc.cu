@@ -20,7 +20,7 @@
 // ranges. Each query block has its own softmax warpgroup; with the 16x32bx2
 // access shape a warp reads 16 rows, threads t and t+16 sharing a row
 // (columns 0-31 and 32-63).
-//   warp 0 / 2  : loader for slot 0 / 1 (lane 0 Q, lane 1 K, lane 2 V; TMA)
+//   warp 0 / 2  : TMA loader for slot 0 / 1 (one thread)
 //   warp 1 / 3  : MMA issuer for slot 0 / 1 (one thread)
 //   warps 4-11  : softmax + epilogue of slot 0 (4-7 block A, 8-11 block B)
 //   warps 12-19 : softmax + epilogue of slot 1
@@ -117,7 +117,7 @@ __device__ __forceinline__ uint64_t global_ns() {
 
 // Bounded wait for the phase of parity `parity`. Returns false if the CTA is
 // aborting or the wait expired (which starts the abort and flags a timeout).
-__device__ __noinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile int *abort_flag,
+__device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile int *abort_flag,
                                       uint32_t *status) {
     if (mbar_try_wait(b, parity)) return true;
     const uint64_t t0 = global_ns();
@@ -138,7 +138,7 @@ __device__ __forceinline__ bool wait_fast(uint64_t *b, uint32_t parity, volatile
     return mbar_try_wait(b, parity) || wait_bar(b, parity, abort_flag, status);
 }
 // Drain wait used on the abort path only: bounded, ignores the abort flag.
-__device__ __noinline__ void drain_bar(uint64_t *b, uint32_t parity) {
+__device__ __forceinline__ void drain_bar(uint64_t *b, uint32_t parity) {
     const uint64_t t0 = global_ns();
     while (!mbar_try_wait(b, parity))
         if (global_ns() - t0 > kDrainNs) return;
@@ -195,6 +195,18 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// max of 32 values as a shallow tree (depth 4) of 3-input maxima
+__device__ __forceinline__ float max32(const float *s) {
+    float a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = fmaxf(fmax3(s[4 * i], s[4 * i + 1], s[4 * i + 2]), s[4 * i + 3]);
+    return fmax3(fmax3(a[0], a[1], a[2]), fmax3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;
@@ -253,50 +265,54 @@ __device__ __forceinline__ int step_block(const TcParams &p, int64_t slab, int i
 
 // ------------------------------------------------------------------ roles
 
+// One thread issues every copy of its slot in consumption order: the pair's
+// two Q tiles, then for each step the K tiles and the V tiles of A and B.
+// (Separate spinning lanes for Q, K and V in one warp would contend for the
+// warp's issue slots; a single sequence does not.)
 __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUtensorMap *tk,
                             const CUtensorMap *tv, SlotTiles &S, SlotBars &B, int slot, int lane,
                             volatile int *abort_flag) {
-    if (lane > 2) return;
+    if (lane != 0) return;
     const int L = 2 * p.w + 1, T = L + p.n;
-    const int64_t first = 2 * (int64_t)blockIdx.x + slot, stride = 2 * (int64_t)gridDim.x;
-    uint32_t c = 0, g = 0;                 // pairs / steps issued by this lane
-    uint64_t *last_bar[2] = {nullptr, nullptr};
-    uint32_t last_par[2] = {0, 0};
+    const int64_t stride = 2 * (int64_t)gridDim.x;
+    uint32_t c = 0, g = 0;                 // pairs / steps issued
+    uint64_t *last_bar[3] = {nullptr, nullptr, nullptr};   // Q, K, V: most recent copy
+    uint32_t last_par[3] = {0, 0, 0};
     bool ok = true;
-    for (int64_t pr = first; pr < p.total_pairs && ok; pr += stride, ++c) {
+    for (int64_t pr = 2 * (int64_t)blockIdx.x + slot; pr < p.total_pairs && ok; pr += stride, ++c) {
         const Pair P = pair_of(p, pr);
         const int64_t base = P.slab * p.n_tokens;
-        if (lane == 0) {                   // Q tiles of the pair (double buffered)
-            const int qb = c & 1;
-            if (!(ok = wait_bar(&B.q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status))) break;
-            mbar_expect_tx(&B.q_full[qb], 2 * TILE);
-            tma_load_tile(S.q[qb][0], tq, &B.q_full[qb], (int)(base + (int64_t)P.iA * BK));
-            tma_load_tile(S.q[qb][1], tq, &B.q_full[qb], (int)(base + (int64_t)P.iB * BK));
-            last_bar[c & 1] = &B.q_full[qb];
-            last_par[c & 1] = (c >> 1) & 1;
-            continue;
-        }
-        for (int t = 0; t < T; ++t, ++g) { // K (lane 1) or V (lane 2) tiles of every step
+        const int qb = c & 1;              // Q tiles of the pair (double buffered)
+        if (!(ok = wait_fast(&B.q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+        mbar_expect_tx(&B.q_full[qb], 2 * TILE);
+        tma_load_tile(S.q[qb][0], tq, &B.q_full[qb], (int)(base + (int64_t)P.iA * BK));
+        tma_load_tile(S.q[qb][1], tq, &B.q_full[qb], (int)(base + (int64_t)P.iB * BK));
+        last_bar[0] = &B.q_full[qb];
+        last_par[0] = (c >> 1) & 1;
+        for (int t = 0; t < T; ++t, ++g) {
             bool va, vb;
             const int ja = step_block(p, P.slab, P.iA, t, va);
             const int jb = step_block(p, P.slab, P.iB, t, vb);
-            if (lane == 1 && t < p.n && (!va || !vb) && p.status) atomicOr(p.status, kStatusBadIndex);
+            if (t < p.n && (!va || !vb) && p.status) atomicOr(p.status, kStatusBadIndex);
             const int st = g & 1;
-            uint64_t *full = lane == 1 ? &B.k_full[st] : &B.v_full[st];
-            uint64_t *empty = lane == 1 ? &B.k_empty[st] : &B.v_empty[st];
-            uint8_t(*dst)[TILE] = lane == 1 ? S.k[st] : S.v[st];
-            const CUtensorMap *map = lane == 1 ? tk : tv;
-            if (!(ok = wait_bar(empty, ((g >> 1) & 1) ^ 1, abort_flag, p.status))) break;
-            if (lane == 2 && (int64_t)g == p.withhold_v_step && blockIdx.x == 0 && slot == 0) continue;
-            mbar_expect_tx(full, 2 * TILE);
-            tma_load_tile(dst[0], map, full, (int)(base + (int64_t)ja * BK));
-            tma_load_tile(dst[1], map, full, (int)(base + (int64_t)jb * BK));
-            last_bar[g & 1] = full;
-            last_par[g & 1] = (g >> 1) & 1;
+            const uint32_t par = ((g >> 1) & 1) ^ 1;
+            if (!(ok = wait_fast(&B.k_empty[st], par, abort_flag, p.status))) break;
+            mbar_expect_tx(&B.k_full[st], 2 * TILE);
+            tma_load_tile(S.k[st][0], tk, &B.k_full[st], (int)(base + (int64_t)ja * BK));
+            tma_load_tile(S.k[st][1], tk, &B.k_full[st], (int)(base + (int64_t)jb * BK));
+            last_bar[1] = &B.k_full[st];
+            last_par[1] = (g >> 1) & 1;
+            if (!(ok = wait_fast(&B.v_empty[st], par, abort_flag, p.status))) break;
+            if ((int64_t)g == p.withhold_v_step && blockIdx.x == 0 && slot == 0) continue;   // test hook
+            mbar_expect_tx(&B.v_full[st], 2 * TILE);
+            tma_load_tile(S.v[st][0], tv, &B.v_full[st], (int)(base + (int64_t)ja * BK));
+            tma_load_tile(S.v[st][1], tv, &B.v_full[st], (int)(base + (int64_t)jb * BK));
+            last_bar[2] = &B.v_full[st];
+            last_par[2] = (g >> 1) & 1;
         }
     }
-    if (!ok) {                             // let copies in flight land before the CTA exits
-        for (int s = 0; s < 2; ++s)
+    if (!ok) {                             // let the copies in flight land before the CTA exits
+        for (int s = 0; s < 3; ++s)
             if (last_bar[s]) drain_bar(last_bar[s], last_par[s]);
     }
 }
@@ -424,11 +440,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             __syncwarp();
             if (lane == 0) mbar_arrive(&B.s_free);
             // ---- softmax numerators against the (lazily updated) running max
-            float mx = -INFINITY;
-            if (valid) {
-#pragma unroll
-                for (int c = 0; c < 32; ++c) mx = fmaxf(mx, s[c]);
-            }
+            float mx = valid ? max32(s) : -INFINITY;
             mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16)) * sl2;
             const bool need = valid && m_used != -INFINITY && mx > m_used + kRescaleLog2;
             const float m_old = m_used;
@@ -436,14 +448,18 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             uint32_t pk[16];
             float ls = 0.f;
             if (valid) {
-                const float nm = -m_used;
+                // p = 2^(s·scale·log2e − m), two columns per packed FMA, four independent sums
+                const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_used, -m_used);
+                float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
-                    const float p0 = ex2(fmaf(s[2 * c], sl2, nm));
-                    const float p1 = ex2(fmaf(s[2 * c + 1], sl2, nm));
-                    pk[c] = pack_bf16(p0, p1);
-                    ls += p0 + p1;
+                    const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
+                    const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                    pk[c] = pack_bf16(e.x, e.y);
+                    acc2[c & 1] = __fadd2_rn(acc2[c & 1], e);
                 }
+                const float2 t2 = __fadd2_rn(acc2[0], acc2[1]);
+                ls = t2.x + t2.y;
             } else {
 #pragma unroll
                 for (int c = 0; c < 16; ++c) pk[c] = 0u;
