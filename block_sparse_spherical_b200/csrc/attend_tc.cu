@@ -20,7 +20,7 @@
 // ranges. Each query block has its own softmax warpgroup; with the 16x32bx2
 // access shape a warp reads 16 rows, threads t and t+16 sharing a row
 // (columns 0-31 and 32-63).
-//   warp 0 / 2  : TMA loader for slot 0 / 1 (one thread)
+//   warp 0 / 2  : TMA loader for slot 0 / 1 (lane 0 issues, the warp holds indices)
 //   warp 1 / 3  : MMA issuer for slot 0 / 1 (one thread)
 //   warps 4-11  : softmax + epilogue of slot 0 (4-7 block A, 8-11 block B)
 //   warps 12-19 : softmax + epilogue of slot 1
@@ -265,53 +265,109 @@ __device__ __forceinline__ int step_block(const TcParams &p, int64_t slab, int i
 
 // ------------------------------------------------------------------ roles
 
-// One thread issues every copy of its slot in consumption order: the pair's
-// two Q tiles, then for each step the K tiles and the V tiles of A and B.
-// (Separate spinning lanes for Q, K and V in one warp would contend for the
-// warp's issue slots; a single sequence does not.)
+// The loader warp issues every copy of its slot from lane 0: the pair's two
+// Q tiles, then K one step ahead of V (K(t+1) before V(t), since S(t+1) is
+// issued before P·V(t)). The other lanes hold the block indices of the
+// current pair (prefetched one pair ahead, so no index load sits on the copy
+// path) and hand them to lane 0 by shuffle.
+struct PairIdx {
+    int a0, a1, b0, b1;   // lane l: selected block l and l+32 of query blocks A and B
+};
+__device__ __forceinline__ PairIdx load_pair_idx(const TcParams &p, int64_t pr, int lane) {
+    PairIdx r{0, 0, 0, 0};
+    if (pr < p.total_pairs) {
+        const Pair P = pair_of(p, pr);
+        const int32_t *ia = p.idx + (P.slab * p.m + P.iA) * (int64_t)p.n;
+        const int32_t *ib = p.idx + (P.slab * p.m + P.iB) * (int64_t)p.n;
+        if (lane < p.n) { r.a0 = __ldg(ia + lane); r.b0 = __ldg(ib + lane); }
+        if (lane + 32 < p.n) { r.a1 = __ldg(ia + lane + 32); r.b1 = __ldg(ib + lane + 32); }
+    }
+    return r;
+}
+
 __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUtensorMap *tk,
                             const CUtensorMap *tv, SlotTiles &S, SlotBars &B, int slot, int lane,
                             volatile int *abort_flag) {
-    if (lane != 0) return;
+    const unsigned FULL = 0xffffffffu;
     const int L = 2 * p.w + 1, T = L + p.n;
     const int64_t stride = 2 * (int64_t)gridDim.x;
-    uint32_t c = 0, g = 0;                 // pairs / steps issued
+    uint32_t c = 0, gk = 0, gv = 0;        // pairs / K steps / V steps issued
     uint64_t *last_bar[3] = {nullptr, nullptr, nullptr};   // Q, K, V: most recent copy
     uint32_t last_par[3] = {0, 0, 0};
     bool ok = true;
-    for (int64_t pr = 2 * (int64_t)blockIdx.x + slot; pr < p.total_pairs && ok; pr += stride, ++c) {
+    int64_t pr = 2 * (int64_t)blockIdx.x + slot;
+    PairIdx cur = load_pair_idx(p, pr, lane);
+    for (; pr < p.total_pairs && ok; pr += stride, ++c) {
+        const PairIdx nxt = load_pair_idx(p, pr + stride, lane);   // in flight during this pair
         const Pair P = pair_of(p, pr);
         const int64_t base = P.slab * p.n_tokens;
-        const int qb = c & 1;              // Q tiles of the pair (double buffered)
-        if (!(ok = wait_fast(&B.q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status))) break;
-        mbar_expect_tx(&B.q_full[qb], 2 * TILE);
-        tma_load_tile(S.q[qb][0], tq, &B.q_full[qb], (int)(base + (int64_t)P.iA * BK));
-        tma_load_tile(S.q[qb][1], tq, &B.q_full[qb], (int)(base + (int64_t)P.iB * BK));
-        last_bar[0] = &B.q_full[qb];
-        last_par[0] = (c >> 1) & 1;
-        for (int t = 0; t < T; ++t, ++g) {
+        // key block of step t for query block i (selected blocks first, then the window)
+        auto block_of = [&](int t, int i, int r0, int r1, bool &valid) -> int {
+            const int js = __shfl_sync(FULL, (t & 32) ? r1 : r0, t & 31);
+            const int j = t < p.n ? js : i - p.w + (t - p.n);
+            valid = j >= 0 && j < p.m;
+            return valid ? j : i;
+        };
+        auto issue_k = [&](int t) -> bool {
             bool va, vb;
-            const int ja = step_block(p, P.slab, P.iA, t, va);
-            const int jb = step_block(p, P.slab, P.iB, t, vb);
-            if (t < p.n && (!va || !vb) && p.status) atomicOr(p.status, kStatusBadIndex);
-            const int st = g & 1;
-            const uint32_t par = ((g >> 1) & 1) ^ 1;
-            if (!(ok = wait_fast(&B.k_empty[st], par, abort_flag, p.status))) break;
-            mbar_expect_tx(&B.k_full[st], 2 * TILE);
-            tma_load_tile(S.k[st][0], tk, &B.k_full[st], (int)(base + (int64_t)ja * BK));
-            tma_load_tile(S.k[st][1], tk, &B.k_full[st], (int)(base + (int64_t)jb * BK));
-            last_bar[1] = &B.k_full[st];
-            last_par[1] = (g >> 1) & 1;
-            if (!(ok = wait_fast(&B.v_empty[st], par, abort_flag, p.status))) break;
-            if ((int64_t)g == p.withhold_v_step && blockIdx.x == 0 && slot == 0) continue;   // test hook
-            mbar_expect_tx(&B.v_full[st], 2 * TILE);
-            tma_load_tile(S.v[st][0], tv, &B.v_full[st], (int)(base + (int64_t)ja * BK));
-            tma_load_tile(S.v[st][1], tv, &B.v_full[st], (int)(base + (int64_t)jb * BK));
-            last_bar[2] = &B.v_full[st];
-            last_par[2] = (g >> 1) & 1;
+            const int ja = block_of(t, P.iA, cur.a0, cur.a1, va);
+            const int jb = block_of(t, P.iB, cur.b0, cur.b1, vb);
+            bool res = true;
+            if (lane == 0) {
+                if (t < p.n && (!va || !vb) && p.status) atomicOr(p.status, kStatusBadIndex);
+                const int st = gk & 1;
+                res = wait_fast(&B.k_empty[st], ((gk >> 1) & 1) ^ 1, abort_flag, p.status);
+                if (res) {
+                    mbar_expect_tx(&B.k_full[st], 2 * TILE);
+                    tma_load_tile(S.k[st][0], tk, &B.k_full[st], (int)(base + (int64_t)ja * BK));
+                    tma_load_tile(S.k[st][1], tk, &B.k_full[st], (int)(base + (int64_t)jb * BK));
+                    last_bar[1] = &B.k_full[st];
+                    last_par[1] = (gk >> 1) & 1;
+                }
+            }
+            ++gk;
+            return __shfl_sync(FULL, res, 0);
+        };
+        auto issue_v = [&](int t) -> bool {
+            bool va, vb;
+            const int ja = block_of(t, P.iA, cur.a0, cur.a1, va);
+            const int jb = block_of(t, P.iB, cur.b0, cur.b1, vb);
+            bool res = true;
+            if (lane == 0) {
+                const int st = gv & 1;
+                res = wait_fast(&B.v_empty[st], ((gv >> 1) & 1) ^ 1, abort_flag, p.status);
+                if (res && !((int64_t)gv == p.withhold_v_step && blockIdx.x == 0 && slot == 0)) {  // test hook
+                    mbar_expect_tx(&B.v_full[st], 2 * TILE);
+                    tma_load_tile(S.v[st][0], tv, &B.v_full[st], (int)(base + (int64_t)ja * BK));
+                    tma_load_tile(S.v[st][1], tv, &B.v_full[st], (int)(base + (int64_t)jb * BK));
+                    last_bar[2] = &B.v_full[st];
+                    last_par[2] = (gv >> 1) & 1;
+                }
+            }
+            ++gv;
+            return __shfl_sync(FULL, res, 0);
+        };
+        bool res = true;
+        if (lane == 0) {                   // Q tiles of the pair (double buffered)
+            const int qb = c & 1;
+            res = wait_fast(&B.q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status);
+            if (res) {
+                mbar_expect_tx(&B.q_full[qb], 2 * TILE);
+                tma_load_tile(S.q[qb][0], tq, &B.q_full[qb], (int)(base + (int64_t)P.iA * BK));
+                tma_load_tile(S.q[qb][1], tq, &B.q_full[qb], (int)(base + (int64_t)P.iB * BK));
+                last_bar[0] = &B.q_full[qb];
+                last_par[0] = (c >> 1) & 1;
+            }
         }
+        if (!(ok = __shfl_sync(FULL, res, 0))) break;
+        if (!(ok = issue_k(0))) break;
+        for (int t = 0; t < T; ++t) {
+            if (t + 1 < T && !(ok = issue_k(t + 1))) break;
+            if (!(ok = issue_v(t))) break;
+        }
+        cur = nxt;
     }
-    if (!ok) {                             // let the copies in flight land before the CTA exits
+    if (!ok && lane == 0) {                // let the copies in flight land before the CTA exits
         for (int s = 0; s < 3; ++s)
             if (last_bar[s]) drain_bar(last_bar[s], last_par[s]);
     }
@@ -394,6 +450,16 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
         const bool mine = wait_fast(b, par, abort_flag, p.status);
         return __all_sync(FULL, mine);
     };
+    int j0 = 0, j1 = 0;                    // this lane's two selected indices of the next pair
+    {
+        const int64_t pr0 = 2 * (int64_t)blockIdx.x + slot;
+        if (pr0 < p.total_pairs) {
+            const Pair P0 = pair_of(p, pr0);
+            const int32_t *ix = p.idx + (P0.slab * p.m + (half ? P0.iB : P0.iA)) * (int64_t)p.n;
+            if (lane < p.n) j0 = __ldg(ix + lane);
+            if (lane + 32 < p.n) j1 = __ldg(ix + lane + 32);
+        }
+    }
     for (int64_t pr = 2 * (int64_t)blockIdx.x + slot; pr < p.total_pairs && ok; pr += stride) {
         const Pair P = pair_of(p, pr);
         const int i = half ? P.iB : P.iA;
@@ -404,14 +470,20 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
         const float *ocg = p.o_cg + (P.slab * p.m + i) * (int64_t)HD + 32 * ch;
         asm volatile("prefetch.global.L1 [%0];" ::"l"(ocg));
         // validity of the n selected blocks of this query block, as a bit mask
-        uint64_t selmask;
+        // (its indices were fetched during the previous pair)
+        const unsigned lo = __ballot_sync(FULL, j0 >= 0 && j0 < p.m);
+        const unsigned hi = __ballot_sync(FULL, j1 >= 0 && j1 < p.m);
+        const uint64_t selmask = ((uint64_t)hi << 32) | lo;
         {
-            const int32_t *ix = p.idx + (P.slab * p.m + i) * (int64_t)p.n;
-            const int j0 = lane < p.n ? __ldg(ix + lane) : 0;
-            const int j1 = lane + 32 < p.n ? __ldg(ix + lane + 32) : 0;
-            const unsigned lo = __ballot_sync(FULL, j0 >= 0 && j0 < p.m);
-            const unsigned hi = __ballot_sync(FULL, j1 >= 0 && j1 < p.m);
-            selmask = ((uint64_t)hi << 32) | lo;
+            const int64_t prn = pr + stride;
+            j0 = j1 = 0;
+            if (prn < p.total_pairs) {
+                const Pair Pn = pair_of(p, prn);
+                const int in = half ? Pn.iB : Pn.iA;
+                const int32_t *ix = p.idx + (Pn.slab * p.m + in) * (int64_t)p.n;
+                if (lane < p.n) j0 = __ldg(ix + lane);
+                if (lane + 32 < p.n) j1 = __ldg(ix + lane + 32);
+            }
         }
         float acc[32];
         float m_used = -INFINITY, l_run = 0.f, l_sel = 0.f;
