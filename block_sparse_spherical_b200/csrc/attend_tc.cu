@@ -13,17 +13,18 @@
 // selection branch reuses the same TMEM accumulator; the epilogue adds
 // g_FG·o_FG and stores bf16.
 //
-// Organisation: a persistent grid of one CTA per SM, 640 threads, two
-// independent pipelines ("slots") per CTA. A slot works on a pair of
-// neighbouring query blocks (A, B) at a time; their M=64 accumulators live
-// in TMEM lanes 0-15 of each 32-lane sub-partition at adjacent 64-column
-// ranges. Each query block has its own softmax warpgroup; with the 16x32bx2
-// access shape a warp reads 16 rows, threads t and t+16 sharing a row
-// (columns 0-31 and 32-63).
-//   warp 0 / 2  : TMA loader for slot 0 / 1 (lane 0 issues, the warp holds indices)
-//   warp 1 / 3  : MMA issuer for slot 0 / 1 (one thread)
-//   warps 4-11  : softmax + epilogue of slot 0 (4-7 block A, 8-11 block B)
-//   warps 12-19 : softmax + epilogue of slot 1
+// Organisation: a persistent grid of one CTA per SM, 640 threads, four
+// independent pipelines ("slots") per CTA, each working on one query block at
+// a time. A slot's M=64 accumulators (S, then O) live in TMEM lanes 0-15 of
+// each 32-lane sub-partition, in its own 128-column range. Four slots give
+// four concurrent MMA issue streams (a single stream of M=64 N=64 MMAs
+// cannot keep the tensor pipe busy) and let the pipelines drift out of phase
+// so that their softmax phases do not all contend for the exp unit at once.
+//   warp s (0-3)   : control of slot s: lane 0 issues the MMAs, lane 1 the
+//                    TMA copies (Q, then K one step ahead of V)
+//   warps 4+4s..7+4s: softmax + epilogue warpgroup of slot s; with the
+//                    16x32bx2 access shape a warp reads 16 rows, threads t
+//                    and t+16 sharing a row (columns 0-31 and 32-63)
 // Every wait on an mbarrier is bounded (2 s); on expiry the kernel records
 // a timeout in the status word, the other roles stop at their next wait,
 // in-flight copies and MMAs are drained (bounded), TMEM is freed and the
@@ -41,20 +42,20 @@ namespace {
 constexpr int BK = 64;                      // tokens per block
 constexpr int HD = 64;                      // head dim
 constexpr int TILE = BK * HD * 2;           // bytes of one 64x64 bf16 tile
-constexpr int NSLOT = 2;
+constexpr int NSLOT = 4;
 constexpr int NTHREADS = 640;
-constexpr uint32_t TMEM_COLS = 512;         // per slot: S_A, S_B, O_A, O_B (64 columns each)
+constexpr uint32_t TMEM_COLS = 512;         // per slot: S and O, 64 columns each
 constexpr float kRescaleLog2 = 8.0f;        // lazy rescale threshold (factor 256)
 constexpr unsigned long long kWaitNs = 2000000000ull;
 constexpr unsigned long long kDrainNs = 200000000ull;
 
 struct alignas(1024) SlotTiles {
-    uint8_t q[2][2][TILE];   // [buffer][A/B]
-    uint8_t k[2][2][TILE];   // [stage][A/B]
-    uint8_t v[2][2][TILE];   // [stage][A/B]
-    uint8_t p[2][TILE];      // [A/B]
+    uint8_t q[2][TILE];      // [buffer]
+    uint8_t k[2][TILE];      // [stage]
+    uint8_t v[2][TILE];      // [stage]
+    uint8_t p[TILE];
 };
-static_assert(sizeof(SlotTiles) == 14 * TILE, "tile layout");
+static_assert(sizeof(SlotTiles) == 7 * TILE, "tile layout");
 
 struct SlotBars {
     uint64_t q_full[2], q_empty[2];
@@ -77,8 +78,8 @@ struct TcParams {
     __nv_bfloat16 *out;     // [slabs*N][64]
     uint32_t *status;       // nullable
     int64_t n_tokens;
-    int64_t total_pairs;
-    int m, n, w, pairs_per_slab;
+    int64_t total_blocks;   // slabs * m query blocks
+    int m, n, w;
     float scale_log2;
     int64_t withhold_v_step;   // test hook, -1 = off
 };
@@ -235,168 +236,108 @@ constexpr uint32_t kIdescBase = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)
 constexpr uint32_t kIdescS = kIdescBase;
 constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);
 
-// ------------------------------------------------------------ work layout
-
-struct Pair {
-    int64_t slab;
-    int iA, iB;
-    bool validB;
-};
-__device__ __forceinline__ Pair pair_of(const TcParams &p, int64_t pr) {
-    Pair r;
-    r.slab = pr / p.pairs_per_slab;
-    r.iA = (int)(pr - r.slab * p.pairs_per_slab) * 2;
-    r.validB = r.iA + 1 < p.m;
-    r.iB = r.validB ? r.iA + 1 : r.iA;
-    return r;
-}
-// Key block of query block i at step t: the n selected blocks first (t < n),
-// then the local window. Out-of-range blocks are masked (loaded as block i, P = 0).
-__device__ __forceinline__ int step_block(const TcParams &p, int64_t slab, int i, int t, bool &valid) {
-    int j;
-    if (t < p.n) {
-        j = __ldg(p.idx + (slab * p.m + i) * (int64_t)p.n + t);
-    } else {
-        j = i - p.w + (t - p.n);
-    }
-    valid = j >= 0 && j < p.m;
-    return valid ? j : i;
-}
-
 // ------------------------------------------------------------------ roles
 
-// The loader warp issues every copy of its slot from lane 0: the pair's two
-// Q tiles, then K one step ahead of V (K(t+1) before V(t), since S(t+1) is
-// issued before P·V(t)). The other lanes hold the block indices of the
-// current pair (prefetched one pair ahead, so no index load sits on the copy
-// path) and hand them to lane 0 by shuffle.
-struct PairIdx {
-    int a0, a1, b0, b1;   // lane l: selected block l and l+32 of query blocks A and B
-};
-__device__ __forceinline__ PairIdx load_pair_idx(const TcParams &p, int64_t pr, int lane) {
-    PairIdx r{0, 0, 0, 0};
-    if (pr < p.total_pairs) {
-        const Pair P = pair_of(p, pr);
-        const int32_t *ia = p.idx + (P.slab * p.m + P.iA) * (int64_t)p.n;
-        const int32_t *ib = p.idx + (P.slab * p.m + P.iB) * (int64_t)p.n;
-        if (lane < p.n) { r.a0 = __ldg(ia + lane); r.b0 = __ldg(ib + lane); }
-        if (lane + 32 < p.n) { r.a1 = __ldg(ia + lane + 32); r.b1 = __ldg(ib + lane + 32); }
-    }
-    return r;
-}
-
+// Copies of one slot, issued by one thread in consumption order: the query
+// block's Q tile, then K one step ahead of V (K(t+1) before V(t), since S(t+1)
+// is issued before P·V(t)). Step t uses the t-th selected block (t < n), then
+// the window blocks i-w .. i+w; blocks outside [0, m) are loaded as block i
+// and masked by the softmax. Selected indices are fetched two steps ahead.
 __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUtensorMap *tk,
-                            const CUtensorMap *tv, SlotTiles &S, SlotBars &B, int slot, int lane,
+                            const CUtensorMap *tv, SlotTiles &S, SlotBars &B, int slot,
                             volatile int *abort_flag) {
-    const unsigned FULL = 0xffffffffu;
     const int L = 2 * p.w + 1, T = L + p.n;
-    const int64_t stride = 2 * (int64_t)gridDim.x;
-    uint32_t c = 0, gk = 0, gv = 0;        // pairs / K steps / V steps issued
+    const int64_t stride = NSLOT * (int64_t)gridDim.x;
+    uint32_t c = 0, gk = 0, gv = 0;
     uint64_t *last_bar[3] = {nullptr, nullptr, nullptr};   // Q, K, V: most recent copy
     uint32_t last_par[3] = {0, 0, 0};
     bool ok = true;
-    int64_t pr = 2 * (int64_t)blockIdx.x + slot;
-    PairIdx cur = load_pair_idx(p, pr, lane);
-    for (; pr < p.total_pairs && ok; pr += stride, ++c) {
-        const PairIdx nxt = load_pair_idx(p, pr + stride, lane);   // in flight during this pair
-        const Pair P = pair_of(p, pr);
-        const int64_t base = P.slab * p.n_tokens;
-        // key block of step t for query block i (selected blocks first, then the window)
-        auto block_of = [&](int t, int i, int r0, int r1, bool &valid) -> int {
-            const int js = __shfl_sync(FULL, (t & 32) ? r1 : r0, t & 31);
-            const int j = t < p.n ? js : i - p.w + (t - p.n);
-            valid = j >= 0 && j < p.m;
-            return valid ? j : i;
+    for (int64_t qi = NSLOT * (int64_t)blockIdx.x + slot; qi < p.total_blocks && ok; qi += stride, ++c) {
+        const int64_t slab = qi / p.m;
+        const int i = (int)(qi - slab * p.m);
+        const int64_t base = slab * p.n_tokens;
+        const int32_t *ix = p.idx + qi * (int64_t)p.n;
+        auto block_of = [&](int t, int jsel) -> int {
+            const int j = t < p.n ? jsel : i - p.w + (t - p.n);
+            return (j >= 0 && j < p.m) ? j : i;
         };
-        auto issue_k = [&](int t) -> bool {
-            bool va, vb;
-            const int ja = block_of(t, P.iA, cur.a0, cur.a1, va);
-            const int jb = block_of(t, P.iB, cur.b0, cur.b1, vb);
-            bool res = true;
-            if (lane == 0) {
-                if (t < p.n && (!va || !vb) && p.status) atomicOr(p.status, kStatusBadIndex);
-                const int st = gk & 1;
-                res = wait_fast(&B.k_empty[st], ((gk >> 1) & 1) ^ 1, abort_flag, p.status);
-                if (res) {
-                    mbar_expect_tx(&B.k_full[st], 2 * TILE);
-                    tma_load_tile(S.k[st][0], tk, &B.k_full[st], (int)(base + (int64_t)ja * BK));
-                    tma_load_tile(S.k[st][1], tk, &B.k_full[st], (int)(base + (int64_t)jb * BK));
-                    last_bar[1] = &B.k_full[st];
-                    last_par[1] = (gk >> 1) & 1;
-                }
-            }
+        int jq[3];                          // selected indices of steps t, t+1, t+2 (ring)
+        jq[0] = p.n > 0 ? __ldg(ix) : 0;
+        jq[1] = p.n > 1 ? __ldg(ix + 1) : 0;
+        jq[2] = p.n > 2 ? __ldg(ix + 2) : 0;
+        const int qb = c & 1;
+        if (!(ok = wait_fast(&B.q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status))) break;
+        mbar_expect_tx(&B.q_full[qb], TILE);
+        tma_load_tile(S.q[qb], tq, &B.q_full[qb], (int)(base + (int64_t)i * BK));
+        last_bar[0] = &B.q_full[qb];
+        last_par[0] = (c >> 1) & 1;
+        int jv = 0;                         // block of the next V copy
+        auto issue_k = [&](int t, int j) -> bool {
+            if (t < p.n && (j < 0 || j >= p.m) && p.status) atomicOr(p.status, kStatusBadIndex);
+            const int st = gk & 1;
+            if (!wait_fast(&B.k_empty[st], ((gk >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+            mbar_expect_tx(&B.k_full[st], TILE);
+            tma_load_tile(S.k[st], tk, &B.k_full[st], (int)(base + (int64_t)block_of(t, j) * BK));
+            last_bar[1] = &B.k_full[st];
+            last_par[1] = (gk >> 1) & 1;
             ++gk;
-            return __shfl_sync(FULL, res, 0);
+            return true;
         };
-        auto issue_v = [&](int t) -> bool {
-            bool va, vb;
-            const int ja = block_of(t, P.iA, cur.a0, cur.a1, va);
-            const int jb = block_of(t, P.iB, cur.b0, cur.b1, vb);
-            bool res = true;
-            if (lane == 0) {
-                const int st = gv & 1;
-                res = wait_fast(&B.v_empty[st], ((gv >> 1) & 1) ^ 1, abort_flag, p.status);
-                if (res && !((int64_t)gv == p.withhold_v_step && blockIdx.x == 0 && slot == 0)) {  // test hook
-                    mbar_expect_tx(&B.v_full[st], 2 * TILE);
-                    tma_load_tile(S.v[st][0], tv, &B.v_full[st], (int)(base + (int64_t)ja * BK));
-                    tma_load_tile(S.v[st][1], tv, &B.v_full[st], (int)(base + (int64_t)jb * BK));
-                    last_bar[2] = &B.v_full[st];
-                    last_par[2] = (gv >> 1) & 1;
-                }
+        auto issue_v = [&](int t, int j) -> bool {
+            const int st = gv & 1;
+            if (!wait_fast(&B.v_empty[st], ((gv >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+            if (!((int64_t)gv == p.withhold_v_step && blockIdx.x == 0 && slot == 0)) {   // test hook
+                mbar_expect_tx(&B.v_full[st], TILE);
+                tma_load_tile(S.v[st], tv, &B.v_full[st], (int)(base + (int64_t)block_of(t, j) * BK));
+                last_bar[2] = &B.v_full[st];
+                last_par[2] = (gv >> 1) & 1;
             }
             ++gv;
-            return __shfl_sync(FULL, res, 0);
+            return true;
         };
-        bool res = true;
-        if (lane == 0) {                   // Q tiles of the pair (double buffered)
-            const int qb = c & 1;
-            res = wait_fast(&B.q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status);
-            if (res) {
-                mbar_expect_tx(&B.q_full[qb], 2 * TILE);
-                tma_load_tile(S.q[qb][0], tq, &B.q_full[qb], (int)(base + (int64_t)P.iA * BK));
-                tma_load_tile(S.q[qb][1], tq, &B.q_full[qb], (int)(base + (int64_t)P.iB * BK));
-                last_bar[0] = &B.q_full[qb];
-                last_par[0] = (c >> 1) & 1;
-            }
-        }
-        if (!(ok = __shfl_sync(FULL, res, 0))) break;
-        if (!(ok = issue_k(0))) break;
+        if (!(ok = issue_k(0, jq[0]))) break;
+        jv = jq[0];
         for (int t = 0; t < T; ++t) {
-            if (t + 1 < T && !(ok = issue_k(t + 1))) break;
-            if (!(ok = issue_v(t))) break;
+            const int jk = jq[(t + 1) % 3];   // index of step t+1
+            if (t + 3 < p.n) jq[(t + 3) % 3] = __ldg(ix + t + 3);
+            else jq[(t + 3) % 3] = jq[t % 3];
+            // (the slot just refilled held step t's index, already used by K(t) and kept in jv)
+            if (t + 1 < T && !(ok = issue_k(t + 1, jk))) break;
+            if (!(ok = issue_v(t, jv))) break;
+            jv = jk;
         }
-        cur = nxt;
     }
-    if (!ok && lane == 0) {                // let the copies in flight land before the CTA exits
-        for (int s = 0; s < 3; ++s)
-            if (last_bar[s]) drain_bar(last_bar[s], last_par[s]);
+    if (!ok) {                             // let the copies in flight land before the CTA exits
+        for (int s2 = 0; s2 < 3; ++s2)
+            if (last_bar[s2]) drain_bar(last_bar[s2], last_par[s2]);
     }
 }
 
-__device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t tmem_slot, int slot, int lane,
+__device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t tmem_slot, int slot,
                          volatile int *abort_flag) {
-    if (lane != 0) return;
     const int L = 2 * p.w + 1, T = L + p.n;
-    const int64_t stride = 2 * (int64_t)gridDim.x;
-    const uint32_t tS = tmem_slot, tO = tmem_slot + 128;
+    const int64_t stride = NSLOT * (int64_t)gridDim.x;
+    const uint32_t tS = tmem_slot, tO = tmem_slot + 64;
+    // shared-memory descriptors of every operand tile, computed once
+    const uint64_t dq0 = desc_kmajor(S.q[0]), dq1 = desc_kmajor(S.q[1]);
+    const uint64_t dk0 = desc_kmajor(S.k[0]), dk1 = desc_kmajor(S.k[1]);
+    const uint64_t dv0 = desc_mnmajor(S.v[0]), dv1 = desc_mnmajor(S.v[1]);
+    const uint64_t dp = desc_kmajor(S.p);
     uint32_t c = 0, g = 0;
     bool ok = true;
-    for (int64_t pr = 2 * (int64_t)blockIdx.x + slot; pr < p.total_pairs && ok; pr += stride, ++c) {
+    for (int64_t qi = NSLOT * (int64_t)blockIdx.x + slot; qi < p.total_blocks && ok; qi += stride, ++c) {
         const int qb = c & 1;
-        if (!(ok = wait_bar(&B.q_full[qb], (c >> 1) & 1, abort_flag, p.status))) break;
-        // S(gs) = Q·K(gs)ᵀ for both query blocks; needs K loaded and the previous S read out
+        if (!(ok = wait_fast(&B.q_full[qb], (c >> 1) & 1, abort_flag, p.status))) break;
+        const uint64_t dq = qb ? dq1 : dq0;
+        // S(gs) = Q·K(gs)ᵀ; needs K loaded and the previous S read out of TMEM
         auto issue_s = [&](uint32_t gs) -> bool {
             const int ks = gs & 1;
             if (!wait_fast(&B.k_full[ks], (gs >> 1) & 1, abort_flag, p.status)) return false;
             if (gs > 0 && !wait_fast(&B.s_free, (gs - 1) & 1, abort_flag, p.status)) return false;
             tc_fence_after();
+            const uint64_t dk = ks ? dk1 : dk0;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint64_t a = desc_kmajor(S.q[qb][h]);
-                const uint64_t b = desc_kmajor(S.k[ks][h]);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) tc_mma(tS + h * 64, a + 2 * kk, b + 2 * kk, kIdescS, kk > 0);
-            }
+            for (int kk = 0; kk < 4; ++kk) tc_mma(tS, dq + 2 * kk, dk + 2 * kk, kIdescS, kk > 0);
             tc_commit(&B.s_full);
             tc_commit(&B.k_empty[ks]);
             return true;
@@ -412,15 +353,10 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
             if (!(ok = wait_fast(&B.p_full, g & 1, abort_flag, p.status))) break;
             if (!(ok = wait_fast(&B.v_full[vs], (g >> 1) & 1, abort_flag, p.status))) break;
             tc_fence_after();
-            const uint32_t accum = (t == 0 || t == p.n) ? 0u : 1u;   // each branch starts a fresh O
+            const uint32_t acc0 = (t == 0 || t == p.n) ? 0u : 1u;   // each branch starts a fresh O
+            const uint64_t dv = vs ? dv1 : dv0;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint64_t a = desc_kmajor(S.p[h]);
-                const uint64_t b = desc_mnmajor(S.v[vs][h]);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    tc_mma(tO + h * 64, a + 2 * kk, b + 128 * kk, kIdescPV, accum | (kk > 0 ? 1u : 0u));
-            }
+            for (int kk = 0; kk < 4; ++kk) tc_mma(tO, dp + 2 * kk, dv + 128 * kk, kIdescPV, kk ? 1u : acc0);
             tc_commit(&B.o_done);
             tc_commit(&B.v_empty[vs]);
         }
@@ -430,57 +366,53 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
     drain_bar(&B.drain, 0);
 }
 
-// One warpgroup per query block of the pair. Thread (wq, lane): row
-// r = 16*wq + lane%16, columns 32*(lane/16) .. +31 of the block's S and O.
+// Softmax warpgroup of a slot. Thread (wq, lane): row r = 16*wq + lane%16,
+// columns 32*(lane/16) .. +31 of the query block's S and O.
 __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t tmem_slot, int slot,
-                             int half, int wq, int lane, volatile int *abort_flag) {
+                             int wq, int lane, volatile int *abort_flag) {
     const unsigned FULL = 0xffffffffu;
     const int L = 2 * p.w + 1, T = L + p.n;
     const int ch = lane >> 4;              // column half of the row
     const int r = 16 * wq + (lane & 15);   // row within the query block
     const uint32_t tlane = (uint32_t)(32 * wq) << 16;
-    const uint32_t tS = tmem_slot + 64 * half + tlane, tO = tmem_slot + 128 + 64 * half + tlane;
-    uint8_t *prow = S.p[half] + (r >> 3) * 1024 + (r & 7) * 128;
+    const uint32_t tS = tmem_slot + tlane, tO = tmem_slot + 64 + tlane;
+    uint8_t *prow = S.p + (r >> 3) * 1024 + (r & 7) * 128;
     const int sw = r & 7;
     const float sl2 = p.scale_log2;
-    const int64_t stride = 2 * (int64_t)gridDim.x;
+    const int64_t stride = NSLOT * (int64_t)gridDim.x;
     uint32_t g = 0;
     bool ok = true;
     auto wait_all = [&](uint64_t *b, uint32_t par) -> bool {
         const bool mine = wait_fast(b, par, abort_flag, p.status);
         return __all_sync(FULL, mine);
     };
-    int j0 = 0, j1 = 0;                    // this lane's two selected indices of the next pair
+    int j0 = 0, j1 = 0;                    // this lane's two selected indices of the next query block
     {
-        const int64_t pr0 = 2 * (int64_t)blockIdx.x + slot;
-        if (pr0 < p.total_pairs) {
-            const Pair P0 = pair_of(p, pr0);
-            const int32_t *ix = p.idx + (P0.slab * p.m + (half ? P0.iB : P0.iA)) * (int64_t)p.n;
+        const int64_t q0 = NSLOT * (int64_t)blockIdx.x + slot;
+        if (q0 < p.total_blocks) {
+            const int32_t *ix = p.idx + q0 * (int64_t)p.n;
             if (lane < p.n) j0 = __ldg(ix + lane);
             if (lane + 32 < p.n) j1 = __ldg(ix + lane + 32);
         }
     }
-    for (int64_t pr = 2 * (int64_t)blockIdx.x + slot; pr < p.total_pairs && ok; pr += stride) {
-        const Pair P = pair_of(p, pr);
-        const int i = half ? P.iB : P.iA;
-        const bool row_valid = half ? P.validB : true;
-        const int64_t tok = P.slab * p.n_tokens + (int64_t)i * BK + r;
+    for (int64_t qi = NSLOT * (int64_t)blockIdx.x + slot; qi < p.total_blocks && ok; qi += stride) {
+        const int64_t slab = qi / p.m;
+        const int i = (int)(qi - slab * p.m);
+        const int64_t tok = slab * p.n_tokens + (int64_t)i * BK + r;
         const float *gp = p.gates + tok * 3;
         const float g_cg = __ldg(gp), g_fg = __ldg(gp + 1), g_l = __ldg(gp + 2);
-        const float *ocg = p.o_cg + (P.slab * p.m + i) * (int64_t)HD + 32 * ch;
+        const float *ocg = p.o_cg + qi * (int64_t)HD + 32 * ch;
         asm volatile("prefetch.global.L1 [%0];" ::"l"(ocg));
         // validity of the n selected blocks of this query block, as a bit mask
-        // (its indices were fetched during the previous pair)
+        // (its indices were fetched during the previous query block)
         const unsigned lo = __ballot_sync(FULL, j0 >= 0 && j0 < p.m);
         const unsigned hi = __ballot_sync(FULL, j1 >= 0 && j1 < p.m);
         const uint64_t selmask = ((uint64_t)hi << 32) | lo;
         {
-            const int64_t prn = pr + stride;
+            const int64_t qn = qi + stride;
             j0 = j1 = 0;
-            if (prn < p.total_pairs) {
-                const Pair Pn = pair_of(p, prn);
-                const int in = half ? Pn.iB : Pn.iA;
-                const int32_t *ix = p.idx + (Pn.slab * p.m + in) * (int64_t)p.n;
+            if (qn < p.total_blocks) {
+                const int32_t *ix = p.idx + qn * (int64_t)p.n;
                 if (lane < p.n) j0 = __ldg(ix + lane);
                 if (lane + 32 < p.n) j1 = __ldg(ix + lane + 32);
             }
@@ -495,7 +427,6 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 const int j = i - p.w + (t - p.n);
                 valid = j >= 0 && j < p.m;
             }
-            valid = valid && row_valid;
             if (t == p.n) {                    // the local branch starts afresh
                 l_sel = l_run;
                 l_run = 0.f;
@@ -520,7 +451,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             uint32_t pk[16];
             float ls = 0.f;
             if (valid) {
-                // p = 2^(s·scale·log2e − m), two columns per packed FMA, four independent sums
+                // p = 2^(s·scale·log2e − m), two columns per packed FMA, two independent sums
                 const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_used, -m_used);
                 float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
@@ -544,24 +475,24 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 const float l = l_sel + __shfl_xor_sync(FULL, l_sel, 16);
                 const float inv = l > 0.f ? g_fg / l : 0.f;
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
+                for (int cc = 0; cc < 2; ++cc) {
                     float o[16];
-                    tmem_ld16(tO + 16 * c, o);
+                    tmem_ld16(tO + 16 * cc, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) acc[16 * c + e] = fmaf(g_cg, __ldg(ocg + 16 * c + e), o[e] * inv);
+                    for (int e = 0; e < 16; ++e) acc[16 * cc + e] = fmaf(g_cg, __ldg(ocg + 16 * cc + e), o[e] * inv);
                 }
             } else if (__any_sync(FULL, need)) {
                 // rows whose running max grew by more than 2^8: rescale their O and sum
                 const float alpha = need ? ex2(m_old - m_used) : 1.f;
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
+                for (int cc = 0; cc < 2; ++cc) {
                     float o[16];
-                    tmem_ld16(tO + 16 * c, o);
+                    tmem_ld16(tO + 16 * cc, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e) o[e] *= alpha;
-                    tmem_st16(tO + 16 * c, o);
+                    tmem_st16(tO + 16 * cc, o);
                 }
                 tmem_wait_st();
                 l_run *= alpha;
@@ -587,18 +518,16 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
         const float inv = l > 0.f ? g_l / l : 0.f;
         uint4 *d4 = reinterpret_cast<uint4 *>(p.out + tok * HD + 32 * ch);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
             float o[16];
-            tmem_ld16(tO + 16 * c, o);
+            tmem_ld16(tO + 16 * cc, o);
             tmem_wait_ld();
             uint32_t w8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                w8[e] = pack_bf16(fmaf(o[2 * e], inv, acc[16 * c + 2 * e]), fmaf(o[2 * e + 1], inv, acc[16 * c + 2 * e + 1]));
-            if (row_valid) {
-                d4[2 * c] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-                d4[2 * c + 1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
-            }
+                w8[e] = pack_bf16(fmaf(o[2 * e], inv, acc[16 * cc + 2 * e]), fmaf(o[2 * e + 1], inv, acc[16 * cc + 2 * e + 1]));
+            d4[2 * cc] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+            d4[2 * cc + 1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
         }
         tc_fence_before();
     }
@@ -626,8 +555,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
                 mbar_init(&B.v_empty[b], 1);
             }
             mbar_init(&B.s_full, 1);
-            mbar_init(&B.s_free, 8);
-            mbar_init(&B.p_full, 8);
+            mbar_init(&B.s_free, 4);
+            mbar_init(&B.p_full, 4);
             mbar_init(&B.o_done, 1);
             mbar_init(&B.drain, 1);
         }
@@ -645,17 +574,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
 
-    if (warp < 4) {
-        const int slot = warp >> 1;
-        if ((warp & 1) == 0)
-            loader_role(p, &tq, &tk, &tv, sh.tiles[slot], sh.bars[slot], slot, lane, abort_flag);
-        else
-            mma_role(p, sh.tiles[slot], sh.bars[slot], tmem + 256u * slot, slot, lane, abort_flag);
+    if (warp < NSLOT) {
+        const int slot = warp;
+        if (lane == 0)
+            mma_role(p, sh.tiles[slot], sh.bars[slot], tmem + 128u * slot, slot, abort_flag);
+        else if (lane == 1)
+            loader_role(p, &tq, &tk, &tv, sh.tiles[slot], sh.bars[slot], slot, abort_flag);
     } else {
-        const int slot = (warp - 4) >> 3;
-        const int half = ((warp - 4) >> 2) & 1;
-        softmax_role(p, sh.tiles[slot], sh.bars[slot], tmem + 256u * slot, slot, half, warp & 3, lane,
-                     abort_flag);
+        const int slot = (warp - NSLOT) >> 2;
+        softmax_role(p, sh.tiles[slot], sh.bars[slot], tmem + 128u * slot, slot, warp & 3, lane, abort_flag);
     }
     __syncwarp();                          // reconverge role lanes before the CTA barrier
 
@@ -723,13 +650,12 @@ cudaError_t launch_attend_tc(const Problem &pb, const void *q, const void *k, co
     p.m = (int)pb.m;
     p.n = (int)pb.top_n;
     p.w = (int)pb.window;
-    p.pairs_per_slab = (int)((pb.m + 1) / 2);
-    p.total_pairs = pb.slabs * p.pairs_per_slab;
+    p.total_blocks = pb.slabs * pb.m;
     p.scale_log2 = pb.scale * 1.4426950408889634f;
     p.withhold_v_step = pb.withhold_v_step;
     const int sms = sm_count();
     if (sms <= 0) return cudaErrorNotSupported;
-    const int64_t want = (p.total_pairs + NSLOT - 1) / NSLOT;
+    const int64_t want = (p.total_blocks + NSLOT - 1) / NSLOT;
     const int grid = (int)(want < sms ? want : sms);
     const size_t smem = sizeof(SharedStorage) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
