@@ -42,25 +42,32 @@ namespace {
 constexpr int BK = 64;                      // tokens per block
 constexpr int HD = 64;                      // head dim
 constexpr int TILE = BK * HD * 2;           // bytes of one 64x64 bf16 tile
-constexpr int NSLOT = 4;
-constexpr int NTHREADS = 640;
+#ifndef BSA_TC_SLOTS
+#define BSA_TC_SLOTS 4
+#endif
+#ifndef BSA_TC_STAGES
+#define BSA_TC_STAGES 2
+#endif
+constexpr int NSLOT = BSA_TC_SLOTS;        // independent pipelines per CTA
+constexpr int NSTAGE = BSA_TC_STAGES;      // depth of the K and V rings
+constexpr int NTHREADS = 32 * (NSLOT + 4 * NSLOT);
 constexpr uint32_t TMEM_COLS = 512;         // per slot: S and O, 64 columns each
 constexpr float kRescaleLog2 = 8.0f;        // lazy rescale threshold (factor 256)
 constexpr unsigned long long kWaitNs = 2000000000ull;
 constexpr unsigned long long kDrainNs = 200000000ull;
 
 struct alignas(1024) SlotTiles {
-    uint8_t q[2][TILE];      // [buffer]
-    uint8_t k[2][TILE];      // [stage]
-    uint8_t v[2][TILE];      // [stage]
+    uint8_t q[2][TILE];        // [buffer]
+    uint8_t k[NSTAGE][TILE];   // [stage]
+    uint8_t v[NSTAGE][TILE];   // [stage]
     uint8_t p[TILE];
 };
-static_assert(sizeof(SlotTiles) == 7 * TILE, "tile layout");
+static_assert(sizeof(SlotTiles) == (3 + 2 * NSTAGE) * TILE, "tile layout");
 
 struct SlotBars {
     uint64_t q_full[2], q_empty[2];
-    uint64_t k_full[2], k_empty[2];
-    uint64_t v_full[2], v_empty[2];
+    uint64_t k_full[NSTAGE], k_empty[NSTAGE];
+    uint64_t v_full[NSTAGE], v_empty[NSTAGE];
     uint64_t s_full, s_free, p_full, o_done, drain;
 };
 
@@ -274,23 +281,23 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
         int jv = 0;                         // block of the next V copy
         auto issue_k = [&](int t, int j) -> bool {
             if (t < p.n && (j < 0 || j >= p.m) && p.status) atomicOr(p.status, kStatusBadIndex);
-            const int st = gk & 1;
-            if (!wait_fast(&B.k_empty[st], ((gk >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+            const int st = gk % NSTAGE;
+            if (!wait_fast(&B.k_empty[st], ((gk / NSTAGE) & 1) ^ 1, abort_flag, p.status)) return false;
             mbar_expect_tx(&B.k_full[st], TILE);
             tma_load_tile(S.k[st], tk, &B.k_full[st], (int)(base + (int64_t)block_of(t, j) * BK));
             last_bar[1] = &B.k_full[st];
-            last_par[1] = (gk >> 1) & 1;
+            last_par[1] = (gk / NSTAGE) & 1;
             ++gk;
             return true;
         };
         auto issue_v = [&](int t, int j) -> bool {
-            const int st = gv & 1;
-            if (!wait_fast(&B.v_empty[st], ((gv >> 1) & 1) ^ 1, abort_flag, p.status)) return false;
+            const int st = gv % NSTAGE;
+            if (!wait_fast(&B.v_empty[st], ((gv / NSTAGE) & 1) ^ 1, abort_flag, p.status)) return false;
             if (!((int64_t)gv == p.withhold_v_step && blockIdx.x == 0 && slot == 0)) {   // test hook
                 mbar_expect_tx(&B.v_full[st], TILE);
                 tma_load_tile(S.v[st], tv, &B.v_full[st], (int)(base + (int64_t)block_of(t, j) * BK));
                 last_bar[2] = &B.v_full[st];
-                last_par[2] = (gv >> 1) & 1;
+                last_par[2] = (gv / NSTAGE) & 1;
             }
             ++gv;
             return true;
@@ -320,8 +327,7 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
     const uint32_t tS = tmem_slot, tO = tmem_slot + 64;
     // shared-memory descriptors of every operand tile, computed once
     const uint64_t dq0 = desc_kmajor(S.q[0]), dq1 = desc_kmajor(S.q[1]);
-    const uint64_t dk0 = desc_kmajor(S.k[0]), dk1 = desc_kmajor(S.k[1]);
-    const uint64_t dv0 = desc_mnmajor(S.v[0]), dv1 = desc_mnmajor(S.v[1]);
+    const uint64_t dk0 = desc_kmajor(S.k[0]), dv0 = desc_mnmajor(S.v[0]);   // stage s: + s*TILE/16
     const uint64_t dp = desc_kmajor(S.p);
     uint32_t c = 0, g = 0;
     bool ok = true;
@@ -331,11 +337,11 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
         const uint64_t dq = qb ? dq1 : dq0;
         // S(gs) = Q·K(gs)ᵀ; needs K loaded and the previous S read out of TMEM
         auto issue_s = [&](uint32_t gs) -> bool {
-            const int ks = gs & 1;
-            if (!wait_fast(&B.k_full[ks], (gs >> 1) & 1, abort_flag, p.status)) return false;
+            const int ks = gs % NSTAGE;
+            if (!wait_fast(&B.k_full[ks], (gs / NSTAGE) & 1, abort_flag, p.status)) return false;
             if (gs > 0 && !wait_fast(&B.s_free, (gs - 1) & 1, abort_flag, p.status)) return false;
             tc_fence_after();
-            const uint64_t dk = ks ? dk1 : dk0;
+            const uint64_t dk = dk0 + (uint64_t)(ks * (TILE >> 4));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) tc_mma(tS, dq + 2 * kk, dk + 2 * kk, kIdescS, kk > 0);
             tc_commit(&B.s_full);
@@ -349,12 +355,12 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
                 if (!(ok = issue_s(g + 1))) break;
                 if (t + 2 == T) tc_commit(&B.q_empty[qb]);
             }
-            const int vs = g & 1;
+            const int vs = g % NSTAGE;
             if (!(ok = wait_fast(&B.p_full, g & 1, abort_flag, p.status))) break;
-            if (!(ok = wait_fast(&B.v_full[vs], (g >> 1) & 1, abort_flag, p.status))) break;
+            if (!(ok = wait_fast(&B.v_full[vs], (g / NSTAGE) & 1, abort_flag, p.status))) break;
             tc_fence_after();
             const uint32_t acc0 = (t == 0 || t == p.n) ? 0u : 1u;   // each branch starts a fresh O
-            const uint64_t dv = vs ? dv1 : dv0;
+            const uint64_t dv = dv0 + (uint64_t)(vs * (TILE >> 4));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) tc_mma(tO, dp + 2 * kk, dv + 128 * kk, kIdescPV, kk ? 1u : acc0);
             tc_commit(&B.o_done);
@@ -549,6 +555,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
             for (int b = 0; b < 2; ++b) {
                 mbar_init(&B.q_full[b], 1);
                 mbar_init(&B.q_empty[b], 1);
+            }
+            for (int b = 0; b < NSTAGE; ++b) {
                 mbar_init(&B.k_full[b], 1);
                 mbar_init(&B.k_empty[b], 1);
                 mbar_init(&B.v_full[b], 1);
@@ -573,6 +581,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
+    static_assert(128 * NSLOT <= (int)TMEM_COLS, "TMEM columns");
 
     if (warp < NSLOT) {
         const int slot = warp;
