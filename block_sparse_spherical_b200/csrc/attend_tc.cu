@@ -57,18 +57,20 @@ constexpr unsigned long long kWaitNs = 2000000000ull;
 constexpr unsigned long long kDrainNs = 200000000ull;
 
 struct alignas(1024) SlotTiles {
-    uint8_t q[2][TILE];        // [buffer]
+    uint8_t q[TILE];
     uint8_t k[NSTAGE][TILE];   // [stage]
     uint8_t v[NSTAGE][TILE];   // [stage]
-    uint8_t p[TILE];
+    uint8_t p[2][TILE];        // [buffer]: P(g) in buffer g%2
 };
 static_assert(sizeof(SlotTiles) == (3 + 2 * NSTAGE) * TILE, "tile layout");
 
 struct SlotBars {
-    uint64_t q_full[2], q_empty[2];
+    uint64_t q_full, q_empty;
+    uint64_t p_full[2], p_empty[2];
     uint64_t k_full[NSTAGE], k_empty[NSTAGE];
     uint64_t v_full[NSTAGE], v_empty[NSTAGE];
-    uint64_t s_full, s_free, p_full, o_done, drain;
+    uint64_t o_done[2];        // [step % 2]: P·V of that step complete
+    uint64_t s_full, s_free, drain;
 };
 
 struct SharedStorage {
@@ -272,12 +274,12 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
         jq[0] = p.n > 0 ? __ldg(ix) : 0;
         jq[1] = p.n > 1 ? __ldg(ix + 1) : 0;
         jq[2] = p.n > 2 ? __ldg(ix + 2) : 0;
-        const int qb = c & 1;
-        if (!(ok = wait_fast(&B.q_empty[qb], ((c >> 1) & 1) ^ 1, abort_flag, p.status))) break;
-        mbar_expect_tx(&B.q_full[qb], TILE);
-        tma_load_tile(S.q[qb], tq, &B.q_full[qb], (int)(base + (int64_t)i * BK));
-        last_bar[0] = &B.q_full[qb];
-        last_par[0] = (c >> 1) & 1;
+        // Q of this query block (single buffer: freed by the previous block's last S)
+        if (!(ok = wait_fast(&B.q_empty, (c & 1) ^ 1, abort_flag, p.status))) break;
+        mbar_expect_tx(&B.q_full, TILE);
+        tma_load_tile(S.q, tq, &B.q_full, (int)(base + (int64_t)i * BK));
+        last_bar[0] = &B.q_full;
+        last_par[0] = c & 1;
         int jv = 0;                         // block of the next V copy
         auto issue_k = [&](int t, int j) -> bool {
             if (t < p.n && (j < 0 || j >= p.m) && p.status) atomicOr(p.status, kStatusBadIndex);
@@ -326,15 +328,13 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
     const int64_t stride = NSLOT * (int64_t)gridDim.x;
     const uint32_t tS = tmem_slot, tO = tmem_slot + 64;
     // shared-memory descriptors of every operand tile, computed once
-    const uint64_t dq0 = desc_kmajor(S.q[0]), dq1 = desc_kmajor(S.q[1]);
+    const uint64_t dq = desc_kmajor(S.q);
     const uint64_t dk0 = desc_kmajor(S.k[0]), dv0 = desc_mnmajor(S.v[0]);   // stage s: + s*TILE/16
-    const uint64_t dp = desc_kmajor(S.p);
+    const uint64_t dp0 = desc_kmajor(S.p[0]), dp1 = desc_kmajor(S.p[1]);
     uint32_t c = 0, g = 0;
     bool ok = true;
     for (int64_t qi = NSLOT * (int64_t)blockIdx.x + slot; qi < p.total_blocks && ok; qi += stride, ++c) {
-        const int qb = c & 1;
-        if (!(ok = wait_fast(&B.q_full[qb], (c >> 1) & 1, abort_flag, p.status))) break;
-        const uint64_t dq = qb ? dq1 : dq0;
+        if (!(ok = wait_fast(&B.q_full, c & 1, abort_flag, p.status))) break;
         // S(gs) = Q·K(gs)ᵀ; needs K loaded and the previous S read out of TMEM
         auto issue_s = [&](uint32_t gs) -> bool {
             const int ks = gs % NSTAGE;
@@ -349,22 +349,24 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
             return true;
         };
         if (!(ok = issue_s(g))) break;
-        if (T == 1) tc_commit(&B.q_empty[qb]);
+        if (T == 1) tc_commit(&B.q_empty);
         for (int t = 0; t < T; ++t, ++g) {
             if (t + 1 < T) {                       // the next S runs while this step's softmax does
                 if (!(ok = issue_s(g + 1))) break;
-                if (t + 2 == T) tc_commit(&B.q_empty[qb]);
+                if (t + 2 == T) tc_commit(&B.q_empty);
             }
-            const int vs = g % NSTAGE;
-            if (!(ok = wait_fast(&B.p_full, g & 1, abort_flag, p.status))) break;
+            const int vs = g % NSTAGE, pb = g & 1;
+            if (!(ok = wait_fast(&B.p_full[pb], (g >> 1) & 1, abort_flag, p.status))) break;
             if (!(ok = wait_fast(&B.v_full[vs], (g / NSTAGE) & 1, abort_flag, p.status))) break;
             tc_fence_after();
             const uint32_t acc0 = (t == 0 || t == p.n) ? 0u : 1u;   // each branch starts a fresh O
             const uint64_t dv = dv0 + (uint64_t)(vs * (TILE >> 4));
+            const uint64_t dp = pb ? dp1 : dp0;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) tc_mma(tO, dp + 2 * kk, dv + 128 * kk, kIdescPV, kk ? 1u : acc0);
-            tc_commit(&B.o_done);
+            tc_commit(&B.o_done[pb]);
             tc_commit(&B.v_empty[vs]);
+            tc_commit(&B.p_empty[pb]);
         }
     }
     // every MMA this thread issued must be complete before TMEM is freed
@@ -382,7 +384,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
     const int r = 16 * wq + (lane & 15);   // row within the query block
     const uint32_t tlane = (uint32_t)(32 * wq) << 16;
     const uint32_t tS = tmem_slot + tlane, tO = tmem_slot + 64 + tlane;
-    uint8_t *prow = S.p + (r >> 3) * 1024 + (r & 7) * 128;
+    const int prow_off = (r >> 3) * 1024 + (r & 7) * 128;
     const int sw = r & 7;
     const float sl2 = p.scale_log2;
     const int64_t stride = NSLOT * (int64_t)gridDim.x;
@@ -473,8 +475,12 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
 #pragma unroll
                 for (int c = 0; c < 16; ++c) pk[c] = 0u;
             }
-            // ---- the previous P·V must be complete before P or O is touched
-            if (g > 0 && !(ok = wait_all(&B.o_done, (g - 1) & 1))) break;
+            // ---- O is touched only at the branch switch or to rescale: then P·V(g-1)
+            //      must be complete
+            // (S(g) complete implies P·V(g-2) complete: one thread issues both, in order,
+            //  so the two-barrier parity below cannot alias)
+            const bool touch_o = (t == p.n) || __any_sync(FULL, need);
+            if (touch_o && g > 0 && !(ok = wait_all(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1))) break;
             tc_fence_after();
             if (t == p.n) {
                 // close the selection branch: acc = g_CG·o_CG + g_FG·o_FG
@@ -488,7 +494,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
 #pragma unroll
                     for (int e = 0; e < 16; ++e) acc[16 * cc + e] = fmaf(g_cg, __ldg(ocg + 16 * cc + e), o[e] * inv);
                 }
-            } else if (__any_sync(FULL, need)) {
+            } else if (touch_o) {
                 // rows whose running max grew by more than 2^8: rescale their O and sum
                 const float alpha = need ? ex2(m_old - m_used) : 1.f;
 #pragma unroll
@@ -504,7 +510,11 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 l_run *= alpha;
             }
             l_run += ls;
-            // ---- P (this thread's 32 columns of the row) -> shared memory, K-major 128-byte swizzle
+            // ---- P (this thread's 32 columns of the row) -> shared memory buffer g%2,
+            //      K-major 128-byte swizzle, once P·V(g-2) has released that buffer
+            const int pb = g & 1;
+            if (!(ok = wait_all(&B.p_empty[pb], ((g >> 1) & 1) ^ 1))) break;
+            uint8_t *prow = S.p[pb] + prow_off;
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
                 const int chunk = 4 * ch + c4;
@@ -514,11 +524,11 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&B.p_full);
+            if (lane == 0) mbar_arrive(&B.p_full[pb]);
         }
         if (!ok) break;
         // ---- epilogue: out = acc + g_L·o_L
-        if (!(ok = wait_all(&B.o_done, (g - 1) & 1))) break;
+        if (!(ok = wait_all(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1))) break;
         tc_fence_after();
         const float l = l_run + __shfl_xor_sync(FULL, l_run, 16);
         const float inv = l > 0.f ? g_l / l : 0.f;
@@ -552,9 +562,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
         sh.abort_flag = 0;
         for (int s = 0; s < NSLOT; ++s) {
             SlotBars &B = sh.bars[s];
+            mbar_init(&B.q_full, 1);
+            mbar_init(&B.q_empty, 1);
             for (int b = 0; b < 2; ++b) {
-                mbar_init(&B.q_full[b], 1);
-                mbar_init(&B.q_empty[b], 1);
+                mbar_init(&B.p_full[b], 4);
+                mbar_init(&B.p_empty[b], 1);
             }
             for (int b = 0; b < NSTAGE; ++b) {
                 mbar_init(&B.k_full[b], 1);
@@ -562,10 +574,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
                 mbar_init(&B.v_full[b], 1);
                 mbar_init(&B.v_empty[b], 1);
             }
+            mbar_init(&B.o_done[0], 1);
+            mbar_init(&B.o_done[1], 1);
             mbar_init(&B.s_full, 1);
             mbar_init(&B.s_free, 4);
-            mbar_init(&B.p_full, 4);
-            mbar_init(&B.o_done, 1);
             mbar_init(&B.drain, 1);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
