@@ -13,18 +13,21 @@
 // selection branch reuses the same TMEM accumulator; the epilogue adds
 // g_FG·o_FG and stores bf16.
 //
-// Organisation: a persistent grid of one CTA per SM, 640 threads, four
+// Organisation: a persistent grid of one CTA per SM, 768 threads, four
 // independent pipelines ("slots") per CTA, each working on one query block at
 // a time. A slot's M=64 accumulators (S, then O) live in TMEM lanes 0-15 of
 // each 32-lane sub-partition, in its own 128-column range. Four slots give
 // four concurrent MMA issue streams (a single stream of M=64 N=64 MMAs
 // cannot keep the tensor pipe busy) and let the pipelines drift out of phase
 // so that their softmax phases do not all contend for the exp unit at once.
-//   warp s (0-3)   : control of slot s: lane 0 issues the MMAs, lane 1 the
-//                    TMA copies (Q, then K one step ahead of V)
-//   warps 4+4s..7+4s: softmax + epilogue warpgroup of slot s; with the
-//                    16x32bx2 access shape a warp reads 16 rows, threads t
-//                    and t+16 sharing a row (columns 0-31 and 32-63)
+//   warp s (0-3)       : MMA issuer of slot s (one thread)
+//   warp 4+s           : TMA loader of slot s (one thread): Q, then K one step
+//                        ahead of V
+//   warps 8+4s..11+4s  : softmax + epilogue warpgroup of slot s; with the
+//                        16x32bx2 access shape a warp reads 16 rows, threads t
+//                        and t+16 sharing a row (columns 0-31 and 32-63)
+// The MMA issuers and the loaders have warps of their own: a lane spinning on
+// one barrier would otherwise hold up the other lane of its warp.
 // Every wait on an mbarrier is bounded (2 s); on expiry the kernel records
 // a timeout in the status word, the other roles stop at their next wait,
 // in-flight copies and MMAs are drained (bounded), TMEM is freed and the
@@ -50,7 +53,12 @@ constexpr int TILE = BK * HD * 2;           // bytes of one 64x64 bf16 tile
 #endif
 constexpr int NSLOT = BSA_TC_SLOTS;        // independent pipelines per CTA
 constexpr int NSTAGE = BSA_TC_STAGES;      // depth of the K and V rings
-constexpr int NTHREADS = 32 * (NSLOT + 4 * NSLOT);
+constexpr int NTHREADS = 32 * (2 * NSLOT + 4 * NSLOT);
+// Register split (setmaxnreg): the two control warpgroups (MMA issuers, loaders)
+// drop to kCtrlRegs, the softmax warpgroups rise to kSoftRegs. The sum must not
+// exceed what the CTA was launched with; the host checks the compiled count.
+constexpr int kCtrlRegs = 40, kSoftRegs = 96;
+constexpr int kRegsNeeded = 2 * NSLOT * 32 * kCtrlRegs + 4 * NSLOT * 32 * kSoftRegs;
 constexpr uint32_t TMEM_COLS = 512;         // per slot: S and O, 64 columns each
 constexpr float kRescaleLog2 = 8.0f;        // lazy rescale threshold (factor 256)
 constexpr unsigned long long kWaitNs = 2000000000ull;
@@ -595,14 +603,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     const uint32_t tmem = sh.tmem_base;
     static_assert(128 * NSLOT <= (int)TMEM_COLS, "TMEM columns");
 
-    if (warp < NSLOT) {
-        const int slot = warp;
-        if (lane == 0)
-            mma_role(p, sh.tiles[slot], sh.bars[slot], tmem + 128u * slot, slot, abort_flag);
-        else if (lane == 1)
-            loader_role(p, &tq, &tk, &tv, sh.tiles[slot], sh.bars[slot], slot, abort_flag);
+    if (warp < 2 * NSLOT) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
+        const int slot = warp % NSLOT;
+        if (warp < NSLOT) {
+            if (lane == 0) mma_role(p, sh.tiles[slot], sh.bars[slot], tmem + 128u * slot, slot, abort_flag);
+        } else {
+            if (lane == 0) loader_role(p, &tq, &tk, &tv, sh.tiles[slot], sh.bars[slot], slot, abort_flag);
+        }
     } else {
-        const int slot = (warp - NSLOT) >> 2;
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
+        const int slot = (warp - 2 * NSLOT) >> 2;
         softmax_role(p, sh.tiles[slot], sh.bars[slot], tmem + 128u * slot, slot, warp & 3, lane, abort_flag);
     }
     __syncwarp();                          // reconverge role lanes before the CTA barrier
@@ -681,6 +692,13 @@ cudaError_t launch_attend_tc(const Problem &pb, const void *q, const void *k, co
     const size_t smem = sizeof(SharedStorage) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    // The register split must fit the registers the CTA is launched with,
+    // otherwise setmaxnreg.inc would wait forever: refuse to launch instead.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, attend_tc_kernel);
+    if (e != cudaSuccess) return e;
+    if ((int64_t)fa.numRegs * NTHREADS < kRegsNeeded || fa.maxThreadsPerBlock < NTHREADS)
+        return cudaErrorInvalidConfiguration;
     attend_tc_kernel<<<grid, NTHREADS, smem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
