@@ -44,6 +44,64 @@ __device__ __forceinline__ bool ranks_above(float av, int ai, float bv, int bi) 
     return av > bv || (av == bv && ai < bi);
 }
 
+// Bitonic sort, within one half-warp, of one row's 64 (logit, block) pairs of
+// the first key tile (4 per lane: element e = 4*tx + r), into the order
+// (logit descending, block ascending). Writes the first 16*NPL of them as the
+// row's initial top list: entry p at lane p%16, slot p/16.
+template <int NPL>
+__device__ __forceinline__ void bitonic_fill(const float *sv, const int *si, int tx, float *lv, int *li) {
+    const unsigned FULL = 0xffffffffu;
+    float v[4];
+    int ix[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) { v[r] = sv[r]; ix[r] = si[r]; }
+#pragma unroll
+    for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j >= 4) {                       // partner in lane tx ^ (j/4), same register
+                const int lj = j >> 2;
+                const bool lower = (tx & lj) == 0;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const bool desc = ((4 * tx + r) & k) == 0;
+                    const float pv = __shfl_xor_sync(FULL, v[r], lj, 16);
+                    const int pi = __shfl_xor_sync(FULL, ix[r], lj, 16);
+                    const bool mine_better = ranks_above(v[r], ix[r], pv, pi);
+                    const bool keep = (lower == desc) ? mine_better : !mine_better;
+                    if (!keep) { v[r] = pv; ix[r] = pi; }
+                }
+            } else {                            // partner in the same lane, register r ^ j
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    if (r & j) continue;
+                    const int r2 = r | j;
+                    const bool desc = ((4 * tx + r) & k) == 0;
+                    const bool b = ranks_above(v[r], ix[r], v[r2], ix[r2]);
+                    if (b != desc) {
+                        const float tv = v[r]; v[r] = v[r2]; v[r2] = tv;
+                        const int ti = ix[r]; ix[r] = ix[r2]; ix[r2] = ti;
+                    }
+                }
+            }
+        }
+    }
+    // rank p (element p) sits in lane p/4, register p%4
+#pragma unroll
+    for (int h = 0; h < NPL; ++h) {
+        const int pr = 16 * h + tx, src = pr >> 2, rr = pr & 3;
+        float c[4];
+        int d[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            c[r] = __shfl_sync(FULL, v[r], src, 16);
+            d[r] = __shfl_sync(FULL, ix[r], src, 16);
+        }
+        lv[h] = rr == 0 ? c[0] : rr == 1 ? c[1] : rr == 2 ? c[2] : c[3];
+        li[h] = rr == 0 ? d[0] : rr == 1 ? d[1] : rr == 2 ? d[2] : d[3];
+    }
+}
+
 template <int D>
 __device__ __forceinline__ void load_rows(float *dst, const float *src, int row0, int m, int tid) {
     // BM rows x D floats -> dst[r*LDS + c], rows >= m zero filled
@@ -148,7 +206,17 @@ compress_select_kernel(const float *__restrict__ qbar, const float *__restrict__
             }
         }
 
-        // ---- top-n merge (rows of this half-warp), candidates in any order
+        // ---- top-n merge (rows of this half-warp)
+        if (t == 0) {
+            // first tile: every logit is a candidate; sort the row's 64 at once
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                int sj[4];
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) sj[jj] = col0 + tx + 16 * jj;
+                bitonic_fill<NPL>(s[i], sj, tx, lv[i], li[i]);
+            }
+        } else
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             float tv = -CUDART_INF_F;
@@ -158,11 +226,16 @@ compress_select_kernel(const float *__restrict__ qbar, const float *__restrict__
                 if (h == hn) { tv = lv[i][h]; ti = li[i][h]; }
             tv = __shfl_sync(FULL, tv, tn, 16);
             ti = __shfl_sync(FULL, ti, tn, 16);
+            // cheap pre-filter (logit >= threshold); the exact (logit, index) order is
+            // applied when the candidate is placed, so ties are still resolved exactly
             unsigned cand = 0;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int j = col0 + tx + 16 * jj;
-                if (j < m && ranks_above(s[i][jj], j, tv, ti)) cand |= 1u << jj;
+            for (int jj = 0; jj < 4; ++jj)
+                if (s[i][jj] >= tv) cand |= 1u << jj;
+            if (col0 + BN > m) {
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj)
+                    if (col0 + tx + 16 * jj >= m) cand &= ~(1u << jj);
             }
             while (__any_sync(FULL, cand != 0)) {
                 const unsigned ball = __ballot_sync(FULL, cand != 0);

@@ -118,3 +118,26 @@ def test_binding_rejects_wrong_tensors():
         bsa(q.transpose(2, 3), k, v, g)
     with pytest.raises(ValueError):
         bsa(q.cpu(), k, v, g)
+
+
+@pytest.mark.parametrize("m,n,d", [(192, 16, 64), (300, 32, 64), (48, 4, 32), (130, 64, 64)])
+def test_selection_ties_exact(m, n, d):
+    """Integer-valued pooled inputs make every logit exact in fp32 and fp64, with many
+    exact ties: the GPU's block lists must equal the oracle's, order included
+    (logit descending, equal logits by lower block index)."""
+    import oracle
+    rng = np.random.default_rng(m * 7 + n)
+    slabs = 2
+    qb = rng.integers(-3, 4, size=(slabs, m, d)).astype(np.float32)
+    kb = rng.integers(-3, 4, size=(slabs, m, d)).astype(np.float32)
+    kb[:, m // 2:] = kb[:, :m - m // 2]          # exact duplicate key blocks
+    vb = rng.standard_normal((slabs, m, d)).astype(np.float32)
+    bs = 16 if d == 32 else 64
+    dt = torch.float32 if d == 32 else torch.bfloat16
+    t = lambda a: torch.from_numpy(a).reshape(1, slabs, m, d).cuda()
+    o_cg, idx = api.compress_select(t(qb), t(kb), t(vb), n, bs, dt)
+    got = idx.cpu().numpy().reshape(slabs, m, n)
+    for s in range(slabs):
+        orc = oracle.compressed_rows(qb[s], kb[s], vb[s], n)
+        assert np.array_equal(got[s], orc["idx"]), f"slab {s}: block lists differ"
+        assert np.max(np.abs(o_cg[0, s].cpu().numpy() - orc["o_cg"])) <= parity.FP32_TOL
