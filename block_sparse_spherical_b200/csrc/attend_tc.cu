@@ -63,6 +63,7 @@ constexpr uint32_t TMEM_COLS = 512;         // per slot: S and O, 64 columns eac
 constexpr float kRescaleLog2 = 8.0f;        // lazy rescale threshold (factor 256)
 constexpr unsigned long long kWaitNs = 2000000000ull;
 constexpr unsigned long long kDrainNs = 200000000ull;
+constexpr uint32_t kSleepNs = 20000;        // suspend hint of a waiting thread (woken at completion)
 
 struct alignas(1024) SlotTiles {
     uint8_t q[TILE];
@@ -127,6 +128,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Same, but a thread whose phase is not complete may sleep up to `ns`
+// nanoseconds (it resumes as soon as the phase completes) instead of
+// returning at once: waiting roles then stop taking issue slots from the
+// warps that have work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *b, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(b)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -140,8 +156,8 @@ __device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile 
     if (mbar_try_wait(b, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(b, parity)) return true;
-        if ((it & 63u) == 0) {
+        if (mbar_try_wait_sleep(b, parity, kSleepNs)) return true;
+        if ((it & 7u) == 0) {
             if (*abort_flag) return false;
             if (global_ns() - t0 > kWaitNs) {
                 *abort_flag = 1;
