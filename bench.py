@@ -237,6 +237,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from block_sparse_spherical_b200 import abi, api
+    from block_sparse_spherical_b200.replicas import (barrier, job_tokens_per_step, max_over_ranks,
+                                                      replica_config)
     from block_sparse_spherical_b200.synthetic import make_inputs
 
     torch.cuda.set_device(local_rank)
@@ -246,8 +248,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
     # independent problem per rank: same workload, rank-offset seed
-    rcfg = cfg.with_(seed=cfg.seed + 1000 * rank) if rank else cfg
-    qh, kh, vh, gh = make_inputs(rcfg)
+    qh, kh, vh, gh = make_inputs(replica_config(cfg, rank))
     tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
 
     def host(a):
@@ -290,8 +291,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         gpu_id = None
     sampler = ClockSampler(gpu_id) if rank == 0 else None
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
+    barrier(dev)
     torch.cuda.synchronize(dev)
     if sampler:
         sampler.start()
@@ -300,16 +300,12 @@ def run_ours(args, cfg, rank, world, local_rank):
         step(evs[s])
     torch.cuda.synchronize(dev)
     clocks = sampler.stop() if sampler else None
-    if world > 1:
-        dist.barrier()
+    barrier(dev)
     total_ms = evs[0][0].elapsed_time(evs[-1][3])
     k_ms = {"pool": [e[0].elapsed_time(e[1]) for e in evs],
             "compress_select": [e[1].elapsed_time(e[2]) for e in evs],
             "fine_attention": [e[2].elapsed_time(e[3]) for e in evs]}
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     if abi.bsa_check_status(status, stream) != 0:
         raise RuntimeError("kernel status word reports an error")
 
@@ -330,19 +326,16 @@ def run_ours(args, cfg, rank, world, local_rank):
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize(dev)
-        if world > 1:
-            dist.barrier()
+        barrier(dev)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(e2e_steps):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(dev)
-        te = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        te_ms = max_over_ranks(a.elapsed_time(b), dev)
         h2d = sum(x.numel() * x.element_size() for x in (qp, kp, vp, gp))
-        e2e = {"value": world * e2e_steps * cfg.slabs * cfg.n_tokens / (float(te.item()) / 1e3), "unit": UNIT,
+        e2e = {"value": e2e_steps * job_tokens_per_step(cfg, world) / (te_ms / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": outp.numel() * outp.element_size(),
                "steps": e2e_steps, "api": "api.BSA.__call__ -> bsa_forward (C ABI)"}
         if bsa.check_status() != 0:
@@ -354,9 +347,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         return
 
     peaks, peak_src = load_peaks()
-    tokens_step = cfg.slabs * cfg.n_tokens
     ms_step = total_ms / args.steps
-    value = world * tokens_step / (ms_step / 1e3)
+    value = job_tokens_per_step(cfg, world) / (ms_step / 1e3)
     fine_flops, comp_flops = cfg.fine_flops(), cfg.compressed_flops()
     mean = {kname: statistics.mean(v) for kname, v in k_ms.items()}
     fine_tflops = fine_flops / (mean["fine_attention"] / 1e3) / 1e12
