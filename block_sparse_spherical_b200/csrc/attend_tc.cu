@@ -57,7 +57,7 @@ constexpr int NTHREADS = 32 * (2 * NSLOT + 4 * NSLOT);
 // Register split (setmaxnreg): the two control warpgroups (MMA issuers, loaders)
 // drop to kCtrlRegs, the softmax warpgroups rise to kSoftRegs. The sum must not
 // exceed what the CTA was launched with; the host checks the compiled count.
-constexpr int kCtrlRegs = 40, kSoftRegs = 96;
+constexpr int kCtrlRegs = 48, kSoftRegs = 96;
 constexpr int kRegsNeeded = 2 * NSLOT * 32 * kCtrlRegs + 4 * NSLOT * 32 * kSoftRegs;
 constexpr uint32_t TMEM_COLS = 512;         // per slot: S and O, 64 columns each
 constexpr float kRescaleLog2 = 8.0f;        // lazy rescale threshold (factor 256)
@@ -178,6 +178,17 @@ __device__ __forceinline__ void drain_bar(uint64_t *b, uint32_t parity) {
         if (global_ns() - t0 > kDrainNs) return;
 }
 
+// One lane of a converged warp (the lowest active one) gets true.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 __device__ __forceinline__ void tma_load_tile(void *dst, const CUtensorMap *map, uint64_t *bar, int row) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
@@ -285,6 +296,10 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
     uint64_t *last_bar[3] = {nullptr, nullptr, nullptr};   // Q, K, V: most recent copy
     uint32_t last_par[3] = {0, 0, 0};
     bool ok = true;
+    const bool leader = elect_one();       // issues the copies; the whole warp runs the loop
+    auto wait_w = [&](uint64_t *b, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, wait_fast(b, par, abort_flag, p.status));
+    };
     for (int64_t qi = NSLOT * (int64_t)blockIdx.x + slot; qi < p.total_blocks && ok; qi += stride, ++c) {
         const int64_t slab = qi / p.m;
         const int i = (int)(qi - slab * p.m);
@@ -299,18 +314,24 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
         jq[1] = p.n > 1 ? __ldg(ix + 1) : 0;
         jq[2] = p.n > 2 ? __ldg(ix + 2) : 0;
         // Q of this query block (single buffer: freed by the previous block's last S)
-        if (!(ok = wait_fast(&B.q_empty, (c & 1) ^ 1, abort_flag, p.status))) break;
-        mbar_expect_tx(&B.q_full, TILE);
-        tma_load_tile(S.q, tq, &B.q_full, (int)(base + (int64_t)i * BK));
+        if (!(ok = wait_w(&B.q_empty, (c & 1) ^ 1))) break;
+        if (leader) {
+            mbar_expect_tx(&B.q_full, TILE);
+            tma_load_tile(S.q, tq, &B.q_full, (int)(base + (int64_t)i * BK));
+        }
+        __syncwarp();
         last_bar[0] = &B.q_full;
         last_par[0] = c & 1;
         int jv = 0;                         // block of the next V copy
         auto issue_k = [&](int t, int j) -> bool {
-            if (t < p.n && (j < 0 || j >= p.m) && p.status) atomicOr(p.status, kStatusBadIndex);
+            if (leader && t < p.n && (j < 0 || j >= p.m) && p.status) atomicOr(p.status, kStatusBadIndex);
             const int st = gk % NSTAGE;
-            if (!wait_fast(&B.k_empty[st], ((gk / NSTAGE) & 1) ^ 1, abort_flag, p.status)) return false;
-            mbar_expect_tx(&B.k_full[st], TILE);
-            tma_load_tile(S.k[st], tk, &B.k_full[st], (int)(base + (int64_t)block_of(t, j) * BK));
+            if (!wait_w(&B.k_empty[st], ((gk / NSTAGE) & 1) ^ 1)) return false;
+            if (leader) {
+                mbar_expect_tx(&B.k_full[st], TILE);
+                tma_load_tile(S.k[st], tk, &B.k_full[st], (int)(base + (int64_t)block_of(t, j) * BK));
+            }
+            __syncwarp();
             last_bar[1] = &B.k_full[st];
             last_par[1] = (gk / NSTAGE) & 1;
             ++gk;
@@ -318,10 +339,13 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
         };
         auto issue_v = [&](int t, int j) -> bool {
             const int st = gv % NSTAGE;
-            if (!wait_fast(&B.v_empty[st], ((gv / NSTAGE) & 1) ^ 1, abort_flag, p.status)) return false;
+            if (!wait_w(&B.v_empty[st], ((gv / NSTAGE) & 1) ^ 1)) return false;
             if (!((int64_t)gv == p.withhold_v_step && blockIdx.x == 0 && slot == 0)) {   // test hook
-                mbar_expect_tx(&B.v_full[st], TILE);
-                tma_load_tile(S.v[st], tv, &B.v_full[st], (int)(base + (int64_t)block_of(t, j) * BK));
+                if (leader) {
+                    mbar_expect_tx(&B.v_full[st], TILE);
+                    tma_load_tile(S.v[st], tv, &B.v_full[st], (int)(base + (int64_t)block_of(t, j) * BK));
+                }
+                __syncwarp();
                 last_bar[2] = &B.v_full[st];
                 last_par[2] = (gv / NSTAGE) & 1;
             }
@@ -357,44 +381,55 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
     const uint64_t dp0 = desc_kmajor(S.p[0]), dp1 = desc_kmajor(S.p[1]);
     uint32_t c = 0, g = 0;
     bool ok = true;
+    const bool leader = elect_one();       // issues MMAs and commits; the whole warp runs the loop
+    auto wait_w = [&](uint64_t *b, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, wait_fast(b, par, abort_flag, p.status));
+    };
     for (int64_t qi = NSLOT * (int64_t)blockIdx.x + slot; qi < p.total_blocks && ok; qi += stride, ++c) {
-        if (!(ok = wait_fast(&B.q_full, c & 1, abort_flag, p.status))) break;
+        if (!(ok = wait_w(&B.q_full, c & 1))) break;
         // S(gs) = Q·K(gs)ᵀ; needs K loaded and the previous S read out of TMEM
         auto issue_s = [&](uint32_t gs) -> bool {
             const int ks = gs % NSTAGE;
-            if (!wait_fast(&B.k_full[ks], (gs / NSTAGE) & 1, abort_flag, p.status)) return false;
-            if (gs > 0 && !wait_fast(&B.s_free, (gs - 1) & 1, abort_flag, p.status)) return false;
+            if (!wait_w(&B.k_full[ks], (gs / NSTAGE) & 1)) return false;
+            if (gs > 0 && !wait_w(&B.s_free, (gs - 1) & 1)) return false;
             tc_fence_after();
             const uint64_t dk = dk0 + (uint64_t)(ks * (TILE >> 4));
+            if (leader) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) tc_mma(tS, dq + 2 * kk, dk + 2 * kk, kIdescS, kk > 0);
-            tc_commit(&B.s_full);
-            tc_commit(&B.k_empty[ks]);
+                for (int kk = 0; kk < 4; ++kk) tc_mma(tS, dq + 2 * kk, dk + 2 * kk, kIdescS, kk > 0);
+                tc_commit(&B.s_full);
+                tc_commit(&B.k_empty[ks]);
+            }
+            __syncwarp();
             return true;
         };
         if (!(ok = issue_s(g))) break;
-        if (T == 1) tc_commit(&B.q_empty);
+        if (T == 1 && leader) tc_commit(&B.q_empty);
         for (int t = 0; t < T; ++t, ++g) {
             if (t + 1 < T) {                       // the next S runs while this step's softmax does
                 if (!(ok = issue_s(g + 1))) break;
-                if (t + 2 == T) tc_commit(&B.q_empty);
+                if (t + 2 == T && leader) tc_commit(&B.q_empty);
             }
             const int vs = g % NSTAGE, pb = g & 1;
-            if (!(ok = wait_fast(&B.p_full[pb], (g >> 1) & 1, abort_flag, p.status))) break;
-            if (!(ok = wait_fast(&B.v_full[vs], (g / NSTAGE) & 1, abort_flag, p.status))) break;
+            if (!(ok = wait_w(&B.p_full[pb], (g >> 1) & 1))) break;
+            if (!(ok = wait_w(&B.v_full[vs], (g / NSTAGE) & 1))) break;
             tc_fence_after();
             const uint32_t acc0 = (t == 0 || t == p.n) ? 0u : 1u;   // each branch starts a fresh O
             const uint64_t dv = dv0 + (uint64_t)(vs * (TILE >> 4));
             const uint64_t dp = pb ? dp1 : dp0;
+            if (leader) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) tc_mma(tO, dp + 2 * kk, dv + 128 * kk, kIdescPV, kk ? 1u : acc0);
-            tc_commit(&B.o_done[pb]);
-            tc_commit(&B.v_empty[vs]);
-            tc_commit(&B.p_empty[pb]);
+                for (int kk = 0; kk < 4; ++kk) tc_mma(tO, dp + 2 * kk, dv + 128 * kk, kIdescPV, kk ? 1u : acc0);
+                tc_commit(&B.o_done[pb]);
+                tc_commit(&B.v_empty[vs]);
+                tc_commit(&B.p_empty[pb]);
+            }
+            __syncwarp();
         }
     }
     // every MMA this thread issued must be complete before TMEM is freed
-    tc_commit(&B.drain);
+    if (leader) tc_commit(&B.drain);
+    __syncwarp();
     drain_bar(&B.drain, 0);
 }
 
@@ -622,11 +657,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     if (warp < 2 * NSLOT) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
         const int slot = warp % NSLOT;
-        if (warp < NSLOT) {
-            if (lane == 0) mma_role(p, sh.tiles[slot], sh.bars[slot], tmem + 128u * slot, slot, abort_flag);
-        } else {
-            if (lane == 0) loader_role(p, &tq, &tk, &tv, sh.tiles[slot], sh.bars[slot], slot, abort_flag);
-        }
+        if (warp < NSLOT)
+            mma_role(p, sh.tiles[slot], sh.bars[slot], tmem + 128u * slot, slot, abort_flag);
+        else
+            loader_role(p, &tq, &tk, &tv, sh.tiles[slot], sh.bars[slot], slot, abort_flag);
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
         const int slot = (warp - 2 * NSLOT) >> 2;
