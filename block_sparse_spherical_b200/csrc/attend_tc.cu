@@ -507,8 +507,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             tmem_ld16(tS + 16, s + 16);
             tmem_wait_ld();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&B.s_free);
+            mbar_arrive(&B.s_free);            // every softmax thread arrives (count 128)
             // ---- softmax numerators against the (lazily updated) running max
             float mx = valid ? max32(s) : -INFINITY;
             mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16)) * sl2;
@@ -582,8 +581,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&B.p_full[pb]);
+            mbar_arrive(&B.p_full[pb]);        // every softmax thread arrives (count 128)
         }
         if (!ok) break;
         // ---- epilogue: out = acc + g_L·o_L
@@ -624,7 +622,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
             mbar_init(&B.q_full, 1);
             mbar_init(&B.q_empty, 1);
             for (int b = 0; b < 2; ++b) {
-                mbar_init(&B.p_full[b], 4);
+                mbar_init(&B.p_full[b], 128);
                 mbar_init(&B.p_empty[b], 1);
             }
             for (int b = 0; b < NSTAGE; ++b) {
@@ -636,7 +634,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
             mbar_init(&B.o_done[0], 1);
             mbar_init(&B.o_done[1], 1);
             mbar_init(&B.s_full, 1);
-            mbar_init(&B.s_free, 4);
+            mbar_init(&B.s_free, 128);
             mbar_init(&B.drain, 1);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
