@@ -5,13 +5,16 @@
 // Thanks to the NESTED order every key/value block is one contiguous 8 KB
 // span, so each is a single TMA box (64 rows x 128 B, 128-byte swizzle)
 // copied straight into the layout tcgen05.mma reads. Per query block the
-// kernel streams its 2w+1 local blocks and then its n selected blocks; for
+// kernel streams its n selected blocks and then its 2w+1 local blocks; for
 // each block it runs S = Q·Kᵀ (tcgen05.mma, M=64 N=64 K=64) into TMEM, an
 // online softmax on the CUDA cores, and O += P·V (tcgen05.mma, P from shared
-// memory). The local branch's output is folded into a register accumulator
-// together with the compressed branch (acc = g_CG·o_CG + g_L·o_L) before the
-// selection branch reuses the same TMEM accumulator; the epilogue adds
-// g_FG·o_FG and stores bf16.
+// memory). The selection branch's output is folded, together with the
+// compressed branch, into a per-thread accumulator (acc = g_CG·o_CG +
+// g_FG·o_FG) before the local branch reuses the same TMEM accumulator; the
+// epilogue adds g_L·o_L and stores bf16. acc is held as fp16 pairs under a
+// power-of-two scale per thread that puts its largest entry in [2^14, 2^15)
+// (relative rounding 2^-11, eight times finer than the bf16 output's): in
+// fp32 it would not fit the softmax warps' register budget and would spill.
 //
 // Organisation: a persistent grid of one CTA per SM, 768 threads, four
 // independent pipelines ("slots") per CTA, each working on one query block at
@@ -33,6 +36,7 @@
 // in-flight copies and MMAs are drained (bounded), TMEM is freed and the
 // kernel returns.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -484,7 +488,8 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 if (lane + 32 < p.n) j1 = __ldg(ix + lane + 32);
             }
         }
-        float acc[32];
+        __half2 acc[16];                   // acc / acc_scale, fp16 pairs
+        float acc_scale = 1.f;
         float m_used = -INFINITY, l_run = 0.f, l_sel = 0.f;
         for (int t = 0; t < T; ++t, ++g) {
             bool valid;
@@ -544,14 +549,25 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 // close the selection branch: acc = g_CG·o_CG + g_FG·o_FG
                 const float l = l_sel + __shfl_xor_sync(FULL, l_sel, 16);
                 const float inv = l > 0.f ? g_fg / l : 0.f;
+                float a[32];
+                tmem_ld16(tO, a);
+                tmem_ld16(tO + 16, a + 16);
+                tmem_wait_ld();
+                float amax = 0.f;
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    float o[16];
-                    tmem_ld16(tO + 16 * cc, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) acc[16 * cc + e] = fmaf(g_cg, __ldg(ocg + 16 * cc + e), o[e] * inv);
+                for (int e = 0; e < 32; ++e) {
+                    a[e] = fmaf(g_cg, __ldg(ocg + e), a[e] * inv);
+                    amax = fmaxf(amax, fabsf(a[e]));
                 }
+                // power-of-two scale 2^k that puts this thread's largest |acc| in
+                // [2^14, 2^15): the fp16 copy neither overflows nor goes subnormal
+                // (all-zero or non-finite values are stored unscaled)
+                const int ex = (__float_as_int(amax) >> 23) & 0xff;
+                const int k = (ex == 0 || ex == 255) ? 0 : min(max(ex - 141, -112), 113);
+                acc_scale = __int_as_float((127 + k) << 23);
+                const float down = __int_as_float((127 - k) << 23);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) acc[e] = __floats2half2_rn(a[2 * e] * down, a[2 * e + 1] * down);
             } else if (touch_o) {
                 // rows whose running max grew by more than 2^8: rescale their O and sum
                 const float alpha = need ? ex2(m_old - m_used) : 1.f;
@@ -597,8 +613,10 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             tmem_wait_ld();
             uint32_t w8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-                w8[e] = pack_bf16(fmaf(o[2 * e], inv, acc[16 * cc + 2 * e]), fmaf(o[2 * e + 1], inv, acc[16 * cc + 2 * e + 1]));
+            for (int e = 0; e < 8; ++e) {
+                const float2 a2 = __half22float2(acc[8 * cc + e]);
+                w8[e] = pack_bf16(fmaf(o[2 * e], inv, a2.x * acc_scale), fmaf(o[2 * e + 1], inv, a2.y * acc_scale));
+            }
             d4[2 * cc] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
             d4[2 * cc + 1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
         }

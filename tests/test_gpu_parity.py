@@ -141,3 +141,27 @@ def test_selection_ties_exact(m, n, d):
         orc = oracle.compressed_rows(qb[s], kb[s], vb[s], n)
         assert np.array_equal(got[s], orc["idx"]), f"slab {s}: block lists differ"
         assert np.max(np.abs(o_cg[0, s].cpu().numpy() - orc["o_cg"])) <= parity.FP32_TOL
+
+
+@pytest.mark.parametrize("log2_scale", [20, -20, 100])
+def test_value_magnitude_range(log2_scale):
+    """V scaled by a power of two (exact in bf16, and the selection does not
+    depend on V): the output scaled back meets the bf16 tolerances against the
+    oracle of the unscaled problem, whose result scales exactly. Covers values
+    far outside fp16's range in both directions, which the kernel's per-thread
+    accumulator of the compressed and selection branches must carry."""
+    cfg = CONFIGS["nside32"]
+    q, k, v, g = parity.device_inputs(cfg)
+    f = 2.0 ** log2_scale
+    vs = (v.float() * f).to(torch.bfloat16)
+    assert torch.equal(vs.float() / f, v.float())
+    bsa = api.BSA.from_config(cfg)
+    out = bsa(q, k, vs, g)
+    torch.cuda.synchronize()
+    assert bsa.check_status() == 0
+    back = (out.float() / f).to(torch.float64)
+    assert torch.isfinite(back).all()
+    for s in (0, cfg.slabs - 1):
+        b, h = divmod(s, cfg.heads)
+        gpu = {"idx": parity.to_np(bsa.sel_idx[b, h]), "out": back[b, h].cpu().numpy()}
+        parity.check_slab(cfg, s, gpu, None)
