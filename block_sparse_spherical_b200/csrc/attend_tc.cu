@@ -23,14 +23,15 @@
 // four concurrent MMA issue streams (a single stream of M=64 N=64 MMAs
 // cannot keep the tensor pipe busy) and let the pipelines drift out of phase
 // so that their softmax phases do not all contend for the exp unit at once.
-//   warp s (0-3)       : MMA issuer of slot s (one thread)
-//   warp 4+s           : TMA loader of slot s (one thread): Q, then K one step
-//                        ahead of V
+//   warp s (0-3)       : MMA warp of slot s
+//   warp 4+s           : TMA copy warp of slot s: Q, then K one step ahead of V
 //   warps 8+4s..11+4s  : softmax + epilogue warpgroup of slot s; with the
 //                        16x32bx2 access shape a warp reads 16 rows, threads t
 //                        and t+16 sharing a row (columns 0-31 and 32-63)
-// The MMA issuers and the loaders have warps of their own: a lane spinning on
-// one barrier would otherwise hold up the other lane of its warp.
+// The MMA and copy roles have warps of their own (a lane spinning on one
+// barrier would otherwise hold up another lane of its warp) and run
+// warp-wide, with uniform control flow; one elected lane issues each MMA,
+// commit and copy.
 // Every wait on an mbarrier is bounded (2 s); on expiry the kernel records
 // a timeout in the status word, the other roles stop at their next wait,
 // in-flight copies and MMAs are drained (bounded), TMEM is freed and the
