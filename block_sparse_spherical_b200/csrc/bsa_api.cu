@@ -72,6 +72,15 @@ bsa_status from_cuda(cudaError_t e) {
     return BSA_ERR_CUDA;
 }
 
+// Compressed branch + top-n: the tensor-core kernel where it takes the shape,
+// else the CUDA-core kernel.
+cudaError_t launch_compress(const Problem &p, const float *qbar, const float *kbar, const float *vbar,
+                            float *o_cg, int32_t *idx, uint32_t *status, cudaStream_t stream) {
+    const cudaError_t e = bsa::launch_compress_tc(p, qbar, kbar, vbar, o_cg, idx, status, stream);
+    if (e != cudaErrorNotSupported) return e;
+    return bsa::launch_compress_select(p, qbar, kbar, vbar, o_cg, idx, stream);
+}
+
 cudaError_t launch_fine(const Problem &p, const void *q, const void *k, const void *v,
                         const float *gates, const float *o_cg, const int32_t *idx, void *out,
                         uint32_t *status, cudaStream_t stream) {
@@ -106,7 +115,7 @@ bsa_status bsa_compress_select(const bsa_config *cfg, const float *qbar, const f
     if (!aligned16(qbar) || !aligned16(kbar) || !aligned16(vbar) || !aligned16(o_cg_block) ||
         !aligned16(sel_idx))
         return BSA_ERR_ALIGNMENT;
-    return from_cuda(bsa::launch_compress_select(p, qbar, kbar, vbar, o_cg_block, sel_idx, stream));
+    return from_cuda(launch_compress(p, qbar, kbar, vbar, o_cg_block, sel_idx, nullptr, stream));
 }
 
 bsa_status bsa_fine_attention(const bsa_config *cfg, const void *q, const void *k, const void *v,
@@ -152,7 +161,7 @@ bsa_status bsa_forward(const bsa_config *cfg, const void *q, const void *k, cons
     float *ocg = reinterpret_cast<float *>(ws + L.o_cg);
     int32_t *idx = sel_idx_out ? sel_idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
     cudaError_t e = bsa::launch_pool(p, q, k, v, qbar, kbar, vbar, stream);
-    if (e == cudaSuccess) e = bsa::launch_compress_select(p, qbar, kbar, vbar, ocg, idx, stream);
+    if (e == cudaSuccess) e = launch_compress(p, qbar, kbar, vbar, ocg, idx, status, stream);
     if (e == cudaSuccess) e = launch_fine(p, q, k, v, gates, ocg, idx, out, status, stream);
     return from_cuda(e);
 }
@@ -265,7 +274,7 @@ extern "C" bsa_status bsa_forward_noalloc(const bsa_config *cfg, const void *q, 
     float *ocg = reinterpret_cast<float *>(ws + L.o_cg);
     int32_t *idx = sel_idx_out ? sel_idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
     cudaError_t e = bsa::launch_pool(p, q, k, v, qbar, kbar, vbar, stream);
-    if (e == cudaSuccess) e = bsa::launch_compress_select(p, qbar, kbar, vbar, ocg, idx, stream);
+    if (e == cudaSuccess) e = launch_compress(p, qbar, kbar, vbar, ocg, idx, status_word, stream);
     if (e == cudaSuccess) e = launch_fine(p, q, k, v, gates, ocg, idx, out, status_word, stream);
     return from_cuda(e);
 }

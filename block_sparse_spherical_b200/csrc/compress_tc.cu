@@ -1,0 +1,477 @@
+// Compressed branch (a) and top-n block selection of branch (b), BSA section
+// of the MOSAIC note, on the sm_100a tensor cores with fp32-accurate products:
+//
+//   z_ij = s·q̄_i·k̄_j,   o_cg_i = Σ_j softmax_j(z_ij) v̄_j,
+//   sel_i = top-n blocks j by (z_ij desc, j asc).
+//
+// Three-pass tf32: every fp32 operand x is split as x = x_hi + x_lo (x_hi = x
+// rounded to tf32, x_lo = the remainder rounded to tf32) and a product as
+// a_hi·b_hi + a_hi·b_lo + a_lo·b_hi: three tcgen05.mma passes of kind tf32
+// into one fp32 accumulator in TMEM. The dropped a_lo·b_lo term and the
+// rounding of the remainders leave a relative error of about 2^-21 per
+// product, the order of an fp32 dot product, so the logits that decide the
+// ranking stay far inside its 1e-4 margin. Each tile's P·V is a fresh
+// accumulation of 24 MMAs; the tiles are summed in fp32 registers.
+//
+// One CTA owns 128 query blocks (rows) of one slab and streams the slab's key
+// blocks in tiles of 64 (the m×m logit matrix never leaves the SM):
+//   warps 0-3  : one thread per row (TMEM lane): reads the row's 64 logits of
+//                the tile, updates its sorted top-n list and the online
+//                softmax, stores the row's P in tf32 parts for the P·V MMA and
+//                folds the previous tile's O into its fp32 accumulator
+//   warps 4-7  : converters: read q̄, k̄, v̄ rows (fp32, L2-resident), split them
+//                into tf32 parts and store them in the MMA's 128-byte-swizzled
+//                K-major layout (V transposed: rows are features, keys run
+//                along K); K runs one tile ahead of V
+//   warp 8     : tensor-core warp (one elected lane issues): S(j) = Q·K(j)ᵀ
+//                into TMEM buffer j%2, then O(j-1) = P(j-1)·V(j-1) into TMEM
+//                buffer (j-1)%2
+//   warps 9-11 : complete the third warpgroup (registers are allocated by
+//                whole warpgroups) and only give their registers away
+// The row threads hold the tile's logits, their output row and their top-n
+// list in registers; a register split (setmaxnreg) moves registers to them
+// from the other warps, by whole warpgroups.
+// Every wait on an mbarrier is bounded (2 s); on expiry the CTA records a
+// timeout (when given a status word), writes -1 as its rows' block indices,
+// drains its MMAs and returns.
+#include <math_constants.h>
+
+#include "tc_common.cuh"
+
+namespace bsa {
+namespace {
+
+using namespace tc;
+
+constexpr int BM = 128;                    // query blocks per CTA
+constexpr int BN = 64;                     // key blocks per tile
+constexpr int D = 64;                      // head dim
+constexpr int NTHREADS = 32 * 12;          // three whole warpgroups (see the register split)
+constexpr int RROWS = 128 * 128;           // bytes of one 128-row swizzled region
+constexpr int KROWS = 64 * 128;            // bytes of one 64-row swizzled region
+constexpr uint32_t TMEM_COLS = 256;        // S buffers at columns 0 and 64, O buffers at 128 and 192
+// Register split: the CTA is launched with 168 registers a thread (384
+// threads, one CTA per SM); the row warpgroup rises to kRowRegs, the other
+// two warpgroups drop to kCtlRegs. 128·kRowRegs + 256·kCtlRegs must not exceed
+// 384·168 (the host checks the compiled launch count), or setmaxnreg.inc would
+// wait forever.
+constexpr int kRowRegs = 232, kCtlRegs = 136;
+constexpr int kRegsNeeded = 128 * kRowRegs + 256 * kCtlRegs;
+
+// instruction descriptor: D f32, A and B tf32, both K-major, M = 128, N = 64
+constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(64 >> 3) << 17) |
+                            ((uint32_t)(128 >> 4) << 24);
+
+struct alignas(1024) Smem {
+    uint8_t qhi[2][RROWS], qlo[2][RROWS];           // A of S: row x feature; region c: features 32c..32c+31
+    uint8_t khi[2][2][KROWS], klo[2][2][KROWS];     // B of S, [stage][region]: key x feature
+    uint8_t vhi[2][KROWS], vlo[2][KROWS];           // B of P·V, [region]: feature x key; region c: keys 32c..
+    uint8_t phi[2][RROWS], plo[2][RROWS];           // A of P·V, [region]: row x key
+    uint64_t q_full, k_full[2], k_empty[2], v_full, v_empty;
+    uint64_t s_full[2], s_free[2], p_full, p_empty, o_full[2], o_free[2], drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory of one CTA");
+
+struct Args {
+    const float *q, *k, *v;                // this slab's q̄, k̄, v̄ [m][64]
+    float *o_cg;                           // this slab's [m][64]
+    int32_t *idx;                          // this slab's [m][n]
+    int m;
+    float sl2;                             // s·log2(e)
+    uint32_t *status;                      // nullable
+};
+
+// Split four fp32 values into tf32 parts; store them as one 16-byte chunk each.
+__device__ __forceinline__ void store_split(uint8_t *hi, uint8_t *lo, uint32_t off, float4 x) {
+    float4 h, l;
+    h.x = to_tf32(x.x);
+    h.y = to_tf32(x.y);
+    h.z = to_tf32(x.z);
+    h.w = to_tf32(x.w);
+    l.x = to_tf32(x.x - h.x);
+    l.y = to_tf32(x.y - h.y);
+    l.z = to_tf32(x.z - h.z);
+    l.w = to_tf32(x.w - h.w);
+    *reinterpret_cast<float4 *>(hi + off) = h;
+    *reinterpret_cast<float4 *>(lo + off) = l;
+}
+
+// Rows [row0, row0+NROWS) of a [m][64] fp32 matrix as a K-major operand: row
+// r's features 32c..32c+31 in region c. Rows at or past m are zero.
+// t: this thread's index among the 128 converters.
+template <int NROWS>
+__device__ __forceinline__ void convert_rows(const float *__restrict__ src, int row0, int m, int t, uint8_t *hi0,
+                                             uint8_t *hi1, uint8_t *lo0, uint8_t *lo1) {
+    constexpr int PER = NROWS * 16 / 128;  // float4 per thread
+    float4 x[PER];
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int i = t + 128 * u, r = i >> 4, c4 = i & 15;
+        x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (row0 + r < m) x[u] = __ldg(reinterpret_cast<const float4 *>(src + (int64_t)(row0 + r) * D) + c4);
+    }
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const int i = t + 128 * u, r = i >> 4, c4 = i & 15;
+        store_split(c4 < 8 ? hi0 : hi1, c4 < 8 ? lo0 : lo1, sw128_offset(r, c4 & 7), x[u]);
+    }
+}
+
+// Keys [key0, key0+64) of v̄ [m][64], transposed into the K-major B operand of
+// P·V: row f (feature) holds the 64 keys, region c keys 32c..32c+31. Each
+// thread moves two 4x4 blocks (4 keys x 4 features). Keys past m are zero.
+__device__ __forceinline__ void convert_v(const float *__restrict__ src, int key0, int m, int t, uint8_t *hi0,
+                                          uint8_t *hi1, uint8_t *lo0, uint8_t *lo1) {
+    float4 x[2][4];
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+        const int blk = t + 128 * b, kg = blk >> 4, fg = blk & 15;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            const int key = key0 + 4 * kg + a;
+            x[b][a] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (key < m) x[b][a] = __ldg(reinterpret_cast<const float4 *>(src + (int64_t)key * D) + fg);
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+        const int blk = t + 128 * b, kg = blk >> 4, fg = blk & 15;
+        uint8_t *hi = kg < 8 ? hi0 : hi1, *lo = kg < 8 ? lo0 : lo1;
+        store_split(hi, lo, sw128_offset(4 * fg + 0, kg & 7), make_float4(x[b][0].x, x[b][1].x, x[b][2].x, x[b][3].x));
+        store_split(hi, lo, sw128_offset(4 * fg + 1, kg & 7), make_float4(x[b][0].y, x[b][1].y, x[b][2].y, x[b][3].y));
+        store_split(hi, lo, sw128_offset(4 * fg + 2, kg & 7), make_float4(x[b][0].z, x[b][1].z, x[b][2].z, x[b][3].z));
+        store_split(hi, lo, sw128_offset(4 * fg + 3, kg & 7), make_float4(x[b][0].w, x[b][1].w, x[b][2].w, x[b][3].w));
+    }
+}
+
+__device__ void convert_role(const Args &a, Smem &sh, int t, int row0, int T, volatile int *abort_flag) {
+    auto wait_c = [&](uint64_t *b, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, mbar_try_wait(b, par) || wait_bar(b, par, abort_flag, a.status));
+    };
+    auto make_k = [&](int x) -> bool {     // K(x) into stage x%2 once S(x-2) has read it
+        const int st = x & 1;
+        if (!wait_c(&sh.k_empty[st], ((x >> 1) & 1) ^ 1)) return false;
+        convert_rows<BN>(a.k, x * BN, a.m, t, sh.khi[st][0], sh.khi[st][1], sh.klo[st][0], sh.klo[st][1]);
+        fence_proxy_async();
+        mbar_arrive(&sh.k_full[st]);
+        return true;
+    };
+    for (int h = 0; h < BM; h += 64)       // Q in two halves of 64 rows (fewer registers)
+        convert_rows<64>(a.q, row0 + h, a.m, t, sh.qhi[0] + h * 128, sh.qhi[1] + h * 128, sh.qlo[0] + h * 128,
+                         sh.qlo[1] + h * 128);
+    fence_proxy_async();
+    mbar_arrive(&sh.q_full);
+    if (!make_k(0)) return;
+    for (int j = 0; j < T; ++j) {
+        if (j + 1 < T && !make_k(j + 1)) return;
+        // V(j) once P·V(j-1) has read the single V buffer
+        if (!wait_c(&sh.v_empty, (j & 1) ^ 1)) return;
+        convert_v(a.v, j * BN, a.m, t, sh.vhi[0], sh.vhi[1], sh.vlo[0], sh.vlo[1]);
+        fence_proxy_async();
+        mbar_arrive(&sh.v_full);
+    }
+}
+
+// D = A·Bᵀ in three tf32 passes (hi·hi, hi·lo, lo·hi) over K = 64: 24 MMAs.
+// a*/b*: the two 32-wide K regions of each operand's parts.
+__device__ __forceinline__ void mma_3pass(uint32_t d, const uint8_t *ah0, const uint8_t *ah1, const uint8_t *al0,
+                                          const uint8_t *al1, const uint8_t *bh0, const uint8_t *bh1,
+                                          const uint8_t *bl0, const uint8_t *bl1) {
+    const uint64_t ah[2] = {desc_kmajor_sw128(ah0), desc_kmajor_sw128(ah1)};
+    const uint64_t al[2] = {desc_kmajor_sw128(al0), desc_kmajor_sw128(al1)};
+    const uint64_t bh[2] = {desc_kmajor_sw128(bh0), desc_kmajor_sw128(bh1)};
+    const uint64_t bl[2] = {desc_kmajor_sw128(bl0), desc_kmajor_sw128(bl1)};
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)          // 8 tf32 (32 B) per MMA
+        mma_tf32(d, ah[kk >> 2] + 2 * (kk & 3), bh[kk >> 2] + 2 * (kk & 3), kIdesc, kk > 0);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        mma_tf32(d, ah[kk >> 2] + 2 * (kk & 3), bl[kk >> 2] + 2 * (kk & 3), kIdesc, 1u);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        mma_tf32(d, al[kk >> 2] + 2 * (kk & 3), bh[kk >> 2] + 2 * (kk & 3), kIdesc, 1u);
+}
+
+__device__ void mma_role(const Args &a, Smem &sh, uint32_t tmem, int T, volatile int *abort_flag) {
+    const bool leader = elect_one();
+    auto wait_w = [&](uint64_t *b, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, mbar_try_wait(b, par) || wait_bar(b, par, abort_flag, a.status));
+    };
+    auto issue_pv = [&](int i) -> bool {   // O(i%2) = P(i)·V(i)
+        if (!wait_w(&sh.p_full, i & 1) || !wait_w(&sh.v_full, i & 1) ||
+            !wait_w(&sh.o_free[i & 1], ((i >> 1) & 1) ^ 1))
+            return false;
+        fence_after();
+        if (leader) {
+            mma_3pass(tmem + 128 + 64 * (i & 1), sh.phi[0], sh.phi[1], sh.plo[0], sh.plo[1], sh.vhi[0], sh.vhi[1],
+                      sh.vlo[0], sh.vlo[1]);
+            commit(&sh.o_full[i & 1]);
+            commit(&sh.v_empty);
+            commit(&sh.p_empty);
+        }
+        __syncwarp();
+        return true;
+    };
+    bool ok = wait_w(&sh.q_full, 0);
+    for (int j = 0; ok && j < T; ++j) {
+        const int st = j & 1;
+        if (!(ok = wait_w(&sh.k_full[st], (j >> 1) & 1))) break;
+        if (!(ok = wait_w(&sh.s_free[st], ((j >> 1) & 1) ^ 1))) break;
+        fence_after();
+        if (leader) {
+            mma_3pass(tmem + 64 * st, sh.qhi[0], sh.qhi[1], sh.qlo[0], sh.qlo[1], sh.khi[st][0], sh.khi[st][1],
+                      sh.klo[st][0], sh.klo[st][1]);
+            commit(&sh.s_full[st]);
+            commit(&sh.k_empty[st]);
+        }
+        __syncwarp();
+        if (j > 0 && !(ok = issue_pv(j - 1))) break;
+    }
+    if (ok && T > 0) ok = issue_pv(T - 1);
+    // every MMA this thread issued must be complete before TMEM is freed
+    if (leader) commit(&sh.drain);
+    __syncwarp();
+    drain_bar(&sh.drain, 0);
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Insert (v, j) into the descending list lv/li of NSEL entries. Keys arrive in
+// ascending j, so an equal logit already in the list keeps its place: the
+// strict comparison realises the (z desc, j asc) order.
+template <int NSEL>
+__device__ __forceinline__ void list_insert(float *lv, int *li, float v, int j) {
+#pragma unroll
+    for (int p = NSEL - 1; p > 0; --p) {
+        const bool up = v > lv[p - 1], here = v > lv[p];
+        const float nv = up ? lv[p - 1] : (here ? v : lv[p]);
+        const int ni = up ? li[p - 1] : (here ? j : li[p]);
+        lv[p] = nv;
+        li[p] = ni;
+    }
+    if (v > lv[0]) {
+        lv[0] = v;
+        li[0] = j;
+    }
+}
+
+template <int NSEL>
+__device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter, int lane, int row0, int T,
+                             volatile int *abort_flag) {
+    const int r = 32 * quarter + lane;     // row of the tile = TMEM lane
+    const int row = row0 + r;
+    const uint32_t tl = (uint32_t)(32 * quarter) << 16;
+    auto wait_s = [&](uint64_t *b, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, mbar_try_wait(b, par) || wait_bar(b, par, abort_flag, a.status));
+    };
+    float lv[NSEL];
+    int li[NSEL];
+#pragma unroll
+    for (int p = 0; p < NSEL; ++p) {
+        lv[p] = -CUDART_INF_F;
+        li[p] = 0x7fffffff;
+    }
+    float m_run = -CUDART_INF_F, l_run = 0.f;   // log2-domain running max and sum of this row
+    float m_acc = -CUDART_INF_F;                // max that o is expressed against
+    float m_even = -CUDART_INF_F, m_odd = -CUDART_INF_F;   // the max P(j) was formed against, j even / odd
+    float o[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) o[c] = 0.f;
+    auto fold_o = [&](int i) -> bool {     // o += O(i), rescaled to the newer max
+        if (!wait_s(&sh.o_full[i & 1], (i >> 1) & 1)) return false;
+        fence_after();
+        float part[D];
+        tmem_ld32(tmem + 128 + 64 * (i & 1) + tl, part);
+        tmem_ld32(tmem + 128 + 64 * (i & 1) + 32 + tl, part + 32);
+        tmem_wait_ld();
+        fence_before();
+        mbar_arrive(&sh.o_free[i & 1]);
+        const float m_i = (i & 1) ? m_odd : m_even;
+        const float f = ex2(m_acc - m_i);
+#pragma unroll
+        for (int c = 0; c < D; ++c) o[c] = fmaf(o[c], f, part[c]);
+        m_acc = m_i;
+        return true;
+    };
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+        const int st = j & 1;
+        if (!(ok = wait_s(&sh.s_full[st], (j >> 1) & 1))) break;
+        fence_after();
+        float s[BN];                       // raw logits q̄·k̄ of keys j*64 .. j*64+63
+        tmem_ld32(tmem + 64 * st + tl, s);
+        tmem_ld32(tmem + 64 * st + 32 + tl, s + 32);
+        tmem_wait_ld();
+        fence_before();
+        mbar_arrive(&sh.s_free[st]);
+        const int key0 = j * BN;
+        if (key0 + BN > a.m) {
+#pragma unroll
+            for (int c = 0; c < BN; ++c)
+                if (key0 + c >= a.m) s[c] = -CUDART_INF_F;
+        }
+        // ---- top-n: candidates beat the list's n-th entry; taken in key order
+#pragma unroll
+        for (int g = 0; g < BN / 8; ++g) {
+            const float thr = lv[NSEL - 1];
+            uint32_t cand = 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (s[8 * g + u] > thr) cand |= 1u << u;
+            while (cand) {
+                const int u = __ffs(cand) - 1;
+                cand &= cand - 1;
+                float v = s[8 * g];
+#pragma unroll
+                for (int uu = 1; uu < 8; ++uu)
+                    if (u == uu) v = s[8 * g + uu];
+                if (v > lv[NSEL - 1]) list_insert<NSEL>(lv, li, v, key0 + 8 * g + u);
+            }
+        }
+        // ---- online softmax (log2 domain) of the row
+        float mt = s[0];
+#pragma unroll
+        for (int c = 1; c < BN; ++c) mt = fmaxf(mt, s[c]);
+        const float m_new = fmaxf(m_run, mt * a.sl2);
+        float ls = 0.f;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+            s[c] = ex2(fmaf(s[c], a.sl2, -m_new));
+            ls += s[c];
+        }
+        l_run = fmaf(l_run, ex2(m_run - m_new), ls);
+        m_run = m_new;
+        if (st) m_odd = m_new;
+        else m_even = m_new;
+        // ---- P(j) in tf32 parts, once P·V(j-1) has read the single P buffer
+        if (!(ok = wait_s(&sh.p_empty, (j & 1) ^ 1))) break;
+#pragma unroll
+        for (int g = 0; g < 2; ++g)
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                store_split(sh.phi[g], sh.plo[g], sw128_offset(r, c),
+                            make_float4(s[32 * g + 4 * c], s[32 * g + 4 * c + 1], s[32 * g + 4 * c + 2],
+                                        s[32 * g + 4 * c + 3]));
+        fence_proxy_async();
+        mbar_arrive(&sh.p_full);
+        if (j > 0 && !(ok = fold_o(j - 1))) break;
+    }
+    if (ok && T > 0) ok = fold_o(T - 1);
+    if (row >= a.m) return;
+    int32_t *ix = a.idx + (int64_t)row * NSEL;
+    if (!ok) {                             // aborted: flag the rows for the selection kernel
+#pragma unroll
+        for (int p = 0; p < NSEL; ++p) ix[p] = -1;
+        return;
+    }
+    const float inv = 1.f / l_run;
+    float4 *dst = reinterpret_cast<float4 *>(a.o_cg + (int64_t)row * D);
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c)
+        dst[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv, o[4 * c + 3] * inv);
+    int4 *idst = reinterpret_cast<int4 *>(ix);
+#pragma unroll
+    for (int p = 0; p < NSEL / 4; ++p) idst[p] = make_int4(li[4 * p], li[4 * p + 1], li[4 * p + 2], li[4 * p + 3]);
+}
+
+template <int NSEL>
+__global__ void __launch_bounds__(NTHREADS, 1)
+compress_tc_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar, const float *__restrict__ vbar,
+                   float *__restrict__ o_cg, int32_t *__restrict__ idx, int m, float sl2, uint32_t *status) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &sh = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t slab = blockIdx.y;
+    const int row0 = blockIdx.x * BM;
+    const int T = (m + BN - 1) / BN;
+    Args a;
+    a.q = qbar + slab * (int64_t)m * D;
+    a.k = kbar + slab * (int64_t)m * D;
+    a.v = vbar + slab * (int64_t)m * D;
+    a.o_cg = o_cg + slab * (int64_t)m * D;
+    a.idx = idx + slab * (int64_t)m * NSEL;
+    a.m = m;
+    a.sl2 = sl2;
+    a.status = status;
+    volatile int *abort_flag = &sh.abort_flag;
+
+    if (threadIdx.x == 0) {
+        sh.abort_flag = 0;
+        mbar_init(&sh.q_full, 128);
+        mbar_init(&sh.v_full, 128);
+        mbar_init(&sh.v_empty, 1);
+        mbar_init(&sh.p_full, 128);
+        mbar_init(&sh.p_empty, 1);
+        mbar_init(&sh.drain, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sh.k_full[b], 128);
+            mbar_init(&sh.k_empty[b], 1);
+            mbar_init(&sh.s_full[b], 1);
+            mbar_init(&sh.s_free[b], 128);
+            mbar_init(&sh.o_full[b], 1);
+            mbar_init(&sh.o_free[b], 128);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 8) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(&sh.tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tmem = sh.tmem_base;
+
+    if (warp < 4) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRowRegs));
+        softmax_role<NSEL>(a, sh, tmem, warp, lane, row0, T, abort_flag);
+    } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
+        if (warp < 8)
+            convert_role(a, sh, threadIdx.x - 128, row0, T, abort_flag);
+        else if (warp == 8)
+            mma_role(a, sh, tmem, T, abort_flag);
+    }
+    __syncwarp();
+
+    fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_compress_tc(const Problem &p, const float *qbar, const float *kbar, const float *vbar,
+                               float *o_cg, int32_t *idx, uint32_t *status, cudaStream_t stream) {
+    if (p.head_dim != D || p.top_n != 16) return cudaErrorNotSupported;
+    if (p.m > 0x7fffffffLL / D) return cudaErrorNotSupported;
+    const size_t smem = sizeof(Smem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(compress_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // the register split must fit the registers the CTA is launched with
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, compress_tc_kernel<16>);
+    if (e != cudaSuccess) return e;
+    if ((int64_t)fa.numRegs * NTHREADS < kRegsNeeded || fa.maxThreadsPerBlock < NTHREADS)
+        return cudaErrorInvalidConfiguration;
+    const dim3 grid((unsigned)((p.m + BM - 1) / BM), (unsigned)p.slabs);
+    compress_tc_kernel<16><<<grid, NTHREADS, smem, stream>>>(qbar, kbar, vbar, o_cg, idx, (int)p.m,
+                                                               p.scale * 1.4426950408889634f, status);
+    return cudaGetLastError();
+}
+
+}  // namespace bsa
