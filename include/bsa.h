@@ -87,10 +87,16 @@ BSA_API bsa_status bsa_pool(const bsa_config *cfg, const void *q, const void *k,
                     float *qbar, float *kbar, float *vbar, cudaStream_t stream);
 
 /*
- * Branch (a) and the top-n choice of branch (b) of the BSA section, all in fp32:
+ * Branch (a) and the top-n choice of branch (b) of the BSA section, with
+ * fp32-accurate arithmetic:
  *   z_ij = s·q̄_i·k̄_j,  o_cg_block[i] = Σ_j softmax_j(z_ij) v̄_j,
  *   sel_idx[i] = the top_n blocks j by (z_ij descending, j ascending).
- * The m×m logit matrix is never written to memory.
+ * The m×m logit matrix is never written to memory. For head_dim 64 and
+ * top_n 16 the products run on the tensor cores as three tf32 products each
+ * (operands split into tf32 high and low parts); other shapes use fp32 on the
+ * CUDA cores. The tensor-core kernel bounds every internal wait (2 s); should
+ * one expire, the affected rows get -1 as their block indices (which
+ * bsa_fine_attention then flags as BSA_ERR_INDEX).
  */
 BSA_API bsa_status bsa_compress_select(const bsa_config *cfg, const float *qbar, const float *kbar,
                                const float *vbar, float *o_cg_block, int32_t *sel_idx,
