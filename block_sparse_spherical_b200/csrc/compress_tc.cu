@@ -5,12 +5,13 @@
 //   sel_i = top-n blocks j by (z_ij desc, j asc).
 //
 // Three-pass tf32: every fp32 operand x is split as x = x_hi + x_lo (x_hi = x
-// rounded to tf32, x_lo = the remainder rounded to tf32) and a product as
-// a_hi·b_hi + a_hi·b_lo + a_lo·b_hi: three tcgen05.mma passes of kind tf32
+// with the 13 low mantissa bits cleared, an exact tf32 value; x_lo = x - x_hi,
+// exact in fp32, of which the tensor core reads the tf32 part) and a product
+// as a_hi·b_hi + a_hi·b_lo + a_lo·b_hi: three tcgen05.mma passes of kind tf32
 // into one fp32 accumulator in TMEM. The dropped a_lo·b_lo term and the
-// rounding of the remainders leave a relative error of about 2^-21 per
-// product, the order of an fp32 dot product, so the logits that decide the
-// ranking stay far inside its 1e-4 margin. Each tile's P·V is a fresh
+// truncated low bits of the remainders leave a relative error below 2^-19 per
+// product, so the logits that decide the ranking stay far inside its 1e-4
+// margin. Each tile's P·V is a fresh
 // accumulation of 24 MMAs; the tiles are summed in fp32 registers.
 //
 // One CTA owns 128 query blocks (rows) of one slab and streams the slab's key
@@ -84,17 +85,19 @@ struct Args {
     uint32_t *status;                      // nullable
 };
 
-// Split four fp32 values into tf32 parts; store them as one 16-byte chunk each.
+// Split four fp32 values into a tf32 high part and the fp32 remainder; store
+// them as one 16-byte chunk each.
+__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xffffe000u); }
 __device__ __forceinline__ void store_split(uint8_t *hi, uint8_t *lo, uint32_t off, float4 x) {
     float4 h, l;
-    h.x = to_tf32(x.x);
-    h.y = to_tf32(x.y);
-    h.z = to_tf32(x.z);
-    h.w = to_tf32(x.w);
-    l.x = to_tf32(x.x - h.x);
-    l.y = to_tf32(x.y - h.y);
-    l.z = to_tf32(x.z - h.z);
-    l.w = to_tf32(x.w - h.w);
+    h.x = tf32_hi(x.x);
+    h.y = tf32_hi(x.y);
+    h.z = tf32_hi(x.z);
+    h.w = tf32_hi(x.w);
+    l.x = x.x - h.x;
+    l.y = x.y - h.y;
+    l.z = x.z - h.z;
+    l.w = x.w - h.w;
     *reinterpret_cast<float4 *>(hi + off) = h;
     *reinterpret_cast<float4 *>(lo + off) = l;
 }
@@ -128,7 +131,7 @@ __device__ __forceinline__ void convert_v(const float *__restrict__ src, int key
     float4 x[2][4];
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-        const int blk = t + 128 * b, kg = blk >> 4, fg = blk & 15;
+        const int blk = t + 128 * b, kg = blk & 15, fg = blk >> 4;   // key group fastest: conflict-free stores
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
             const int key = key0 + 4 * kg + a;
@@ -138,7 +141,7 @@ __device__ __forceinline__ void convert_v(const float *__restrict__ src, int key
     }
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-        const int blk = t + 128 * b, kg = blk >> 4, fg = blk & 15;
+        const int blk = t + 128 * b, kg = blk & 15, fg = blk >> 4;
         uint8_t *hi = kg < 8 ? hi0 : hi1, *lo = kg < 8 ? lo0 : lo1;
         store_split(hi, lo, sw128_offset(4 * fg + 0, kg & 7), make_float4(x[b][0].x, x[b][1].x, x[b][2].x, x[b][3].x));
         store_split(hi, lo, sw128_offset(4 * fg + 1, kg & 7), make_float4(x[b][0].y, x[b][1].y, x[b][2].y, x[b][3].y));
@@ -243,6 +246,37 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// lv/li = the first NSEL entries of s (keys 0..NSEL-1) sorted by (value
+// descending, key ascending): a bitonic network on registers.
+template <int NSEL>
+__device__ __forceinline__ void sort_desc(const float *s, float *lv, int *li) {
+#pragma unroll
+    for (int p = 0; p < NSEL; ++p) {
+        lv[p] = s[p];
+        li[p] = p;
+    }
+#pragma unroll
+    for (int k = 2; k <= NSEL; k <<= 1)
+#pragma unroll
+        for (int jj = k >> 1; jj > 0; jj >>= 1)
+#pragma unroll
+            for (int p = 0; p < NSEL; ++p) {
+                const int q = p ^ jj;
+                if (q <= p) continue;
+                // (p, q) in descending order within ascending-k blocks of alternating direction
+                const bool desc = (p & k) == 0;
+                const bool q_above = lv[q] > lv[p] || (lv[q] == lv[p] && li[q] < li[p]);
+                if (q_above == desc) {
+                    const float tv = lv[p];
+                    lv[p] = lv[q];
+                    lv[q] = tv;
+                    const int ti = li[p];
+                    li[p] = li[q];
+                    li[q] = ti;
+                }
+            }
+}
+
 // Insert (v, j) into the descending list lv/li of NSEL entries. Keys arrive in
 // ascending j, so an equal logit already in the list keeps its place: the
 // strict comparison realises the (z desc, j asc) order.
@@ -317,9 +351,16 @@ __device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter
             for (int c = 0; c < BN; ++c)
                 if (key0 + c >= a.m) s[c] = -CUDART_INF_F;
         }
-        // ---- top-n: candidates beat the list's n-th entry; taken in key order
+        // ---- top-n: candidates beat the list's n-th entry; taken in key order.
+        //      The first tile seeds the list with its first NSEL logits, sorted.
+        int g0 = 0;
+        if (j == 0) {
+            sort_desc<NSEL>(s, lv, li);
+            g0 = NSEL / 8;
+        }
 #pragma unroll
         for (int g = 0; g < BN / 8; ++g) {
+            if (g < g0) continue;
             const float thr = lv[NSEL - 1];
             uint32_t cand = 0;
 #pragma unroll
