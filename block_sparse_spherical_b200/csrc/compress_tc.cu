@@ -240,6 +240,11 @@ __device__ void mma_role(const Args &a, Smem &sh, uint32_t tmem, int T, volatile
     drain_bar(&sh.drain, 0);
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -358,10 +363,16 @@ __device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter
             sort_desc<NSEL>(s, lv, li);
             g0 = NSEL / 8;
         }
+        float gm[BN / 8];                  // maxima of the 8 groups of 8 logits
+#pragma unroll
+        for (int g = 0; g < BN / 8; ++g)
+            gm[g] = fmax3(fmax3(s[8 * g], s[8 * g + 1], s[8 * g + 2]), fmax3(s[8 * g + 3], s[8 * g + 4], s[8 * g + 5]),
+                          fmaxf(s[8 * g + 6], s[8 * g + 7]));
 #pragma unroll
         for (int g = 0; g < BN / 8; ++g) {
             if (g < g0) continue;
             const float thr = lv[NSEL - 1];
+            if (!(gm[g] > thr)) continue;  // no candidate in this group
             uint32_t cand = 0;
 #pragma unroll
             for (int u = 0; u < 8; ++u)
@@ -377,9 +388,7 @@ __device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter
             }
         }
         // ---- online softmax (log2 domain) of the row
-        float mt = s[0];
-#pragma unroll
-        for (int c = 1; c < BN; ++c) mt = fmaxf(mt, s[c]);
+        const float mt = fmax3(fmax3(gm[0], gm[1], gm[2]), fmax3(gm[3], gm[4], gm[5]), fmaxf(gm[6], gm[7]));
         const float m_new = fmaxf(m_run, mt * a.sl2);
         float ls = 0.f;
 #pragma unroll
