@@ -43,9 +43,12 @@
 #include <mutex>
 
 #include "bsa_internal.cuh"
+#include "tc_common.cuh"
 
 namespace bsa {
 namespace {
+
+using namespace tc;
 
 constexpr int BK = 64;                      // tokens per block
 constexpr int HD = 64;                      // head dim
@@ -66,9 +69,6 @@ constexpr int kCtrlRegs = 48, kSoftRegs = 96;
 constexpr int kRegsNeeded = 2 * NSLOT * 32 * kCtrlRegs + 4 * NSLOT * 32 * kSoftRegs;
 constexpr uint32_t TMEM_COLS = 512;         // per slot: S and O, 64 columns each
 constexpr float kRescaleLog2 = 8.0f;        // lazy rescale threshold (factor 256)
-constexpr unsigned long long kWaitNs = 2000000000ull;
-constexpr unsigned long long kDrainNs = 200000000ull;
-constexpr uint32_t kSleepNs = 20000;        // suspend hint of a waiting thread (woken at completion)
 
 struct alignas(1024) SlotTiles {
     uint8_t q[TILE];
@@ -109,105 +109,6 @@ struct TcParams {
 
 // ---------------------------------------------------------------- PTX glue
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Same, but a thread whose phase is not complete may sleep up to `ns`
-// nanoseconds (it resumes as soon as the phase completes) instead of
-// returning at once: waiting roles then stop taking issue slots from the
-// warps that have work.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *b, uint32_t parity, uint32_t ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity), "r"(ns)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Bounded wait for the phase of parity `parity`. Returns false if the CTA is
-// aborting or the wait expired (which starts the abort and flags a timeout).
-__device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile int *abort_flag,
-                                      uint32_t *status) {
-    if (mbar_try_wait(b, parity)) return true;
-    const uint64_t t0 = global_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait_sleep(b, parity, kSleepNs)) return true;
-        if ((it & 7u) == 0) {
-            if (*abort_flag) return false;
-            if (global_ns() - t0 > kWaitNs) {
-                *abort_flag = 1;
-                if (status) atomicOr(status, kStatusTimeout);
-                return false;
-            }
-        }
-    }
-}
-__device__ __forceinline__ bool wait_fast(uint64_t *b, uint32_t parity, volatile int *abort_flag,
-                                          uint32_t *status) {
-    return mbar_try_wait(b, parity) || wait_bar(b, parity, abort_flag, status);
-}
-// Drain wait used on the abort path only: bounded, ignores the abort flag.
-__device__ __forceinline__ void drain_bar(uint64_t *b, uint32_t parity) {
-    const uint64_t t0 = global_ns();
-    while (!mbar_try_wait(b, parity))
-        if (global_ns() - t0 > kDrainNs) return;
-}
-
-// One lane of a converged warp (the lowest active one) gets true.
-__device__ __forceinline__ bool elect_one() {
-    uint32_t pred;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "elect.sync _|p, 0xffffffff;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(pred));
-    return pred != 0;
-}
-
-__device__ __forceinline__ void tma_load_tile(void *dst, const CUtensorMap *map, uint64_t *bar, int row) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(row)
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
     asm volatile(
@@ -238,20 +139,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *r) {
         "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
         : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-// max of 32 values as a shallow tree (depth 4) of 3-input maxima
 __device__ __forceinline__ float max32(const float *s) {
     float a[8];
 #pragma unroll
@@ -397,43 +285,43 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
             const int ks = gs % NSTAGE;
             if (!wait_w(&B.k_full[ks], (gs / NSTAGE) & 1)) return false;
             if (gs > 0 && !wait_w(&B.s_free, (gs - 1) & 1)) return false;
-            tc_fence_after();
+            fence_after();
             const uint64_t dk = dk0 + (uint64_t)(ks * (TILE >> 4));
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) tc_mma(tS, dq + 2 * kk, dk + 2 * kk, kIdescS, kk > 0);
-                tc_commit(&B.s_full);
-                tc_commit(&B.k_empty[ks]);
+                commit(&B.s_full);
+                commit(&B.k_empty[ks]);
             }
             __syncwarp();
             return true;
         };
         if (!(ok = issue_s(g))) break;
-        if (T == 1 && leader) tc_commit(&B.q_empty);
+        if (T == 1 && leader) commit(&B.q_empty);
         for (int t = 0; t < T; ++t, ++g) {
             if (t + 1 < T) {                       // the next S runs while this step's softmax does
                 if (!(ok = issue_s(g + 1))) break;
-                if (t + 2 == T && leader) tc_commit(&B.q_empty);
+                if (t + 2 == T && leader) commit(&B.q_empty);
             }
             const int vs = g % NSTAGE, pb = g & 1;
             if (!(ok = wait_w(&B.p_full[pb], (g >> 1) & 1))) break;
             if (!(ok = wait_w(&B.v_full[vs], (g / NSTAGE) & 1))) break;
-            tc_fence_after();
+            fence_after();
             const uint32_t acc0 = (t == 0 || t == p.n) ? 0u : 1u;   // each branch starts a fresh O
             const uint64_t dv = dv0 + (uint64_t)(vs * (TILE >> 4));
             const uint64_t dp = pb ? dp1 : dp0;
             if (leader) {
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) tc_mma(tO, dp + 2 * kk, dv + 128 * kk, kIdescPV, kk ? 1u : acc0);
-                tc_commit(&B.o_done[pb]);
-                tc_commit(&B.v_empty[vs]);
-                tc_commit(&B.p_empty[pb]);
+                commit(&B.o_done[pb]);
+                commit(&B.v_empty[vs]);
+                commit(&B.p_empty[pb]);
             }
             __syncwarp();
         }
     }
     // every MMA this thread issued must be complete before TMEM is freed
-    if (leader) tc_commit(&B.drain);
+    if (leader) commit(&B.drain);
     __syncwarp();
     drain_bar(&B.drain, 0);
 }
@@ -507,12 +395,12 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             }
             // ---- scores of this step
             if (!(ok = wait_all(&B.s_full, g & 1))) break;
-            tc_fence_after();
+            fence_after();
             float s[32];
             tmem_ld16(tS, s);
             tmem_ld16(tS + 16, s + 16);
             tmem_wait_ld();
-            tc_fence_before();
+            fence_before();
             mbar_arrive(&B.s_free);            // every softmax thread arrives (count 128)
             // ---- softmax numerators against the (lazily updated) running max
             float mx = valid ? max32(s) : -INFINITY;
@@ -545,7 +433,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             //  so the two-barrier parity below cannot alias)
             const bool touch_o = (t == p.n) || __any_sync(FULL, need);
             if (touch_o && g > 0 && !(ok = wait_all(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1))) break;
-            tc_fence_after();
+            fence_after();
             if (t == p.n) {
                 // close the selection branch: acc = g_CG·o_CG + g_FG·o_FG
                 const float l = l_sel + __shfl_xor_sync(FULL, l_sel, 16);
@@ -597,13 +485,13 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 *reinterpret_cast<uint4 *>(prow + ((chunk ^ sw) << 4)) = v4;
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            tc_fence_before();
+            fence_before();
             mbar_arrive(&B.p_full[pb]);        // every softmax thread arrives (count 128)
         }
         if (!ok) break;
         // ---- epilogue: out = acc + g_L·o_L
         if (!(ok = wait_all(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1))) break;
-        tc_fence_after();
+        fence_after();
         const float l = l_run + __shfl_xor_sync(FULL, l_run, 16);
         const float inv = l > 0.f ? g_l / l : 0.f;
         uint4 *d4 = reinterpret_cast<uint4 *>(p.out + tok * HD + 32 * ch);
@@ -621,7 +509,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             d4[2 * cc] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
             d4[2 * cc + 1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
         }
-        tc_fence_before();
+        fence_before();
     }
 }
 
@@ -665,9 +553,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    tc_fence_before();
+    fence_before();
     __syncthreads();
-    tc_fence_after();
+    fence_after();
     const uint32_t tmem = sh.tmem_base;
     static_assert(128 * NSLOT <= (int)TMEM_COLS, "TMEM columns");
 
@@ -685,10 +573,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     }
     __syncwarp();                          // reconverge role lanes before the CTA barrier
 
-    tc_fence_before();
+    fence_before();
     __syncthreads();
     if (warp == 0) {
-        tc_fence_after();
+        fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
                      : "memory");
     }

@@ -240,16 +240,6 @@ __device__ void mma_role(const Args &a, Smem &sh, uint32_t tmem, int T, volatile
     drain_bar(&sh.drain, 0);
 }
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 // lv/li = the first NSEL entries of s (keys 0..NSEL-1) sorted by (value
 // descending, key ascending): a bitonic network on registers.

@@ -1,8 +1,10 @@
 // Device helpers for the sm_100a tensor-core kernels: mbarriers with bounded
-// waits, tcgen05 fences/commits, TMEM loads, and the 128-byte-swizzled
-// K-major shared-memory operand layout that tcgen05.mma reads.
+// waits, TMA tile copies, tcgen05 fences/commits, TMEM loads, the 128-byte-
+// swizzled K-major shared-memory operand layout that tcgen05.mma reads, and a
+// few arithmetic one-liners.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -21,6 +23,10 @@ __device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t *b) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+                 : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *b, uint32_t parity) {
     uint32_t ok;
@@ -69,6 +75,10 @@ __device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile 
         }
     }
 }
+__device__ __forceinline__ bool wait_fast(uint64_t *b, uint32_t parity, volatile int *abort_flag,
+                                          uint32_t *status) {
+    return mbar_try_wait(b, parity) || wait_bar(b, parity, abort_flag, status);
+}
 // Drain wait used on the abort path only: bounded, ignores the abort flag.
 __device__ __forceinline__ void drain_bar(uint64_t *b, uint32_t parity) {
     const uint64_t t0 = global_ns();
@@ -84,6 +94,15 @@ __device__ __forceinline__ bool elect_one() {
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(pred));
     return pred != 0;
+}
+
+// 2-D TMA tile copy (row coordinate `row`, column 0) completing on `bar`.
+__device__ __forceinline__ void tma_load_tile(void *dst, const CUtensorMap *map, uint64_t *bar, int row) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(0), "r"(row)
+        : "memory");
 }
 
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -118,6 +137,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *r) {
         : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle:
 // rows of 128 B, groups of 8 rows 1024 B apart (start address 16-B units,
@@ -134,11 +154,15 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(const void *tile) {
 // Byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled region.
 __device__ __forceinline__ uint32_t sw128_offset(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
-// fp32 -> tf32 (round to nearest, ties away), returned as an fp32 bit pattern.
-__device__ __forceinline__ float to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 }  // namespace tc
