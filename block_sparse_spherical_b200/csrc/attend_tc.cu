@@ -175,7 +175,7 @@ constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);
 
 // ------------------------------------------------------------------ roles
 
-// Copies of one slot, issued by one thread in consumption order: the query
+// Copies of one slot, issued by the copy warp's elected lane in consumption order: the query
 // block's Q tile, then K one step ahead of V (K(t+1) before V(t), since S(t+1)
 // is issued before P·V(t)). Step t uses the t-th selected block (t < n), then
 // the window blocks i-w .. i+w; blocks outside [0, m) are loaded as block i
