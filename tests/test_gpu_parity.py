@@ -72,7 +72,7 @@ EDGE = {
     "window_covers_all": (64, 64, "bf16", 640, 1, 2, 3, 20),
     "topn_equals_m": (64, 64, "bf16", 2048, 1, 2, 32, 1),
     "tc_compress_n_eq_m16": (64, 64, "bf16", 1024, 1, 2, 16, 1),
-    "tc_compress_m257_two_row_tiles": (64, 64, "bf16", 64 * 257, 1, 3, 16, 2),
+    "tc_compress_m257_ragged": (64, 64, "bf16", 64 * 257, 1, 3, 16, 2),
     "f32_block64": (64, 64, "f32", 4096, 1, 2, 8, 1),
     "f32_tiny_n_eq_m": (16, 32, "f32", 768, 1, 2, 48, 1),
     "f32_tiny_ragged": (16, 32, "f32", 16 * 75, 3, 1, 5, 3),
