@@ -19,8 +19,8 @@ STATUS_NAMES = {
     0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "BSA_ERR_ALIGNMENT",
     4: "BSA_ERR_CUDA", 5: "BSA_ERR_TIMEOUT", 6: "BSA_ERR_WORKSPACE", 7: "BSA_ERR_INDEX",
 }
-EXPORTS = ("bsa_pool", "bsa_compress_select", "bsa_fine_attention", "bsa_workspace_size",
-           "bsa_forward", "bsa_check_status", "bsa_status_string", "bsa_forward_noalloc")
+EXPORTS = ("bsa_pool", "bsa_compress_select", "bsa_compress_select_ws", "bsa_fine_attention",
+           "bsa_workspace_size", "bsa_forward", "bsa_check_status", "bsa_status_string", "bsa_forward_noalloc")
 TESTING_EXPORTS = ("bsa_testing_fine_attention_withhold",)
 
 
@@ -51,6 +51,7 @@ def load() -> ctypes.CDLL:
     sig = {
         "bsa_pool": [C, P, P, P, P, P, P, P],
         "bsa_compress_select": [C, P, P, P, P, P, P],
+        "bsa_compress_select_ws": [C, P, P, P, P, P, P, S, P],
         "bsa_fine_attention": [C, P, P, P, P, P, P, P, P, P],
         "bsa_workspace_size": [C, ctypes.POINTER(ctypes.c_size_t)],
         "bsa_forward": [C, P, P, P, P, P, P, P, S, P],
@@ -102,6 +103,13 @@ def bsa_compress_select(cfg: BsaConfig, qbar, kbar, vbar, o_cg_block, sel_idx, s
     _check("bsa_compress_select", load().bsa_compress_select(
         ctypes.byref(cfg), _ptr(qbar), _ptr(kbar), _ptr(vbar), _ptr(o_cg_block), _ptr(sel_idx),
         _stream(stream)))
+
+
+def bsa_compress_select_ws(cfg: BsaConfig, qbar, kbar, vbar, o_cg_block, sel_idx, workspace, workspace_bytes: int,
+                           stream=None) -> None:
+    _check("bsa_compress_select_ws", load().bsa_compress_select_ws(
+        ctypes.byref(cfg), _ptr(qbar), _ptr(kbar), _ptr(vbar), _ptr(o_cg_block), _ptr(sel_idx),
+        _ptr(workspace), workspace_bytes, _stream(stream)))
 
 
 def bsa_fine_attention(cfg: BsaConfig, q, k, v, gates, o_cg_block, sel_idx, out, status_word=None,

@@ -49,7 +49,10 @@ bsa_status make_problem(const bsa_config *cfg, Problem *p) {
 }
 
 struct WorkspaceLayout {
-    size_t status, qbar, kbar, vbar, o_cg, idx, total;
+    size_t status, qbar, kbar, vbar, o_cg, idx;
+    size_t base;      // end of the above (what the allocation-free entry point needs)
+    size_t split;     // tf32 split images of the tensor-core compressed kernel (0 bytes if unused)
+    size_t total;
 };
 
 WorkspaceLayout layout_of(const Problem &p) {
@@ -62,7 +65,9 @@ WorkspaceLayout layout_of(const Problem &p) {
     w.vbar = w.kbar + round_up(pooled);
     w.o_cg = w.vbar + round_up(pooled);
     w.idx = w.o_cg + round_up(pooled);
-    w.total = w.idx + round_up(idx);
+    w.base = w.idx + round_up(idx);
+    w.split = w.base;
+    w.total = w.split + round_up(bsa::compress_tc_workspace_bytes(p));
     return w;
 }
 
@@ -72,11 +77,11 @@ bsa_status from_cuda(cudaError_t e) {
     return BSA_ERR_CUDA;
 }
 
-// Compressed branch + top-n: the tensor-core kernel where it takes the shape,
-// else the CUDA-core kernel.
+// Compressed branch + top-n: the tensor-core kernel where it takes the shape
+// (with its split images in `images` when given), else the CUDA-core kernel.
 cudaError_t launch_compress(const Problem &p, const float *qbar, const float *kbar, const float *vbar,
-                            float *o_cg, int32_t *idx, uint32_t *status, cudaStream_t stream) {
-    const cudaError_t e = bsa::launch_compress_tc(p, qbar, kbar, vbar, o_cg, idx, status, stream);
+                            float *o_cg, int32_t *idx, uint32_t *status, void *images, cudaStream_t stream) {
+    const cudaError_t e = bsa::launch_compress_tc(p, qbar, kbar, vbar, o_cg, idx, status, images, stream);
     if (e != cudaErrorNotSupported) return e;
     return bsa::launch_compress_select(p, qbar, kbar, vbar, o_cg, idx, stream);
 }
@@ -115,7 +120,24 @@ bsa_status bsa_compress_select(const bsa_config *cfg, const float *qbar, const f
     if (!aligned16(qbar) || !aligned16(kbar) || !aligned16(vbar) || !aligned16(o_cg_block) ||
         !aligned16(sel_idx))
         return BSA_ERR_ALIGNMENT;
-    return from_cuda(launch_compress(p, qbar, kbar, vbar, o_cg_block, sel_idx, nullptr, stream));
+    return from_cuda(launch_compress(p, qbar, kbar, vbar, o_cg_block, sel_idx, nullptr, nullptr, stream));
+}
+
+bsa_status bsa_compress_select_ws(const bsa_config *cfg, const float *qbar, const float *kbar,
+                                  const float *vbar, float *o_cg_block, int32_t *sel_idx, void *workspace,
+                                  size_t workspace_bytes, cudaStream_t stream) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (!qbar || !kbar || !vbar || !o_cg_block || !sel_idx) return BSA_ERR_INVALID_ARG;
+    if (!workspace) return BSA_ERR_WORKSPACE;
+    const WorkspaceLayout L = layout_of(p);
+    if (workspace_bytes < L.total) return BSA_ERR_WORKSPACE;
+    if (!aligned16(qbar) || !aligned16(kbar) || !aligned16(vbar) || !aligned16(o_cg_block) ||
+        !aligned16(sel_idx) || ((uintptr_t)workspace & (kAlign - 1)))
+        return BSA_ERR_ALIGNMENT;
+    void *images = L.total > L.split ? static_cast<char *>(workspace) + L.split : nullptr;
+    return from_cuda(launch_compress(p, qbar, kbar, vbar, o_cg_block, sel_idx, nullptr, images, stream));
 }
 
 bsa_status bsa_fine_attention(const bsa_config *cfg, const void *q, const void *k, const void *v,
@@ -161,7 +183,8 @@ bsa_status bsa_forward(const bsa_config *cfg, const void *q, const void *k, cons
     float *ocg = reinterpret_cast<float *>(ws + L.o_cg);
     int32_t *idx = sel_idx_out ? sel_idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
     cudaError_t e = bsa::launch_pool(p, q, k, v, qbar, kbar, vbar, stream);
-    if (e == cudaSuccess) e = launch_compress(p, qbar, kbar, vbar, ocg, idx, status, stream);
+    void *images = L.total > L.split ? ws + L.split : nullptr;
+    if (e == cudaSuccess) e = launch_compress(p, qbar, kbar, vbar, ocg, idx, status, images, stream);
     if (e == cudaSuccess) e = launch_fine(p, q, k, v, gates, ocg, idx, out, status, stream);
     return from_cuda(e);
 }
@@ -261,7 +284,7 @@ extern "C" bsa_status bsa_forward_noalloc(const bsa_config *cfg, const void *q, 
     if (st != BSA_OK) return st;
     if (!q || !k || !v || !gates || !out) return BSA_ERR_INVALID_ARG;
     const WorkspaceLayout L = layout_of(p);
-    if (L.total > kNoAllocScratchBytes) return BSA_ERR_WORKSPACE;   // problem too large for the fixed scratch
+    if (L.base > kNoAllocScratchBytes) return BSA_ERR_WORKSPACE;    // problem too large for the fixed scratch
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gates) || !aligned16(out) ||
         !aligned16(sel_idx_out) || ((uintptr_t)status_word & 3u))
         return BSA_ERR_ALIGNMENT;
@@ -274,7 +297,7 @@ extern "C" bsa_status bsa_forward_noalloc(const bsa_config *cfg, const void *q, 
     float *ocg = reinterpret_cast<float *>(ws + L.o_cg);
     int32_t *idx = sel_idx_out ? sel_idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
     cudaError_t e = bsa::launch_pool(p, q, k, v, qbar, kbar, vbar, stream);
-    if (e == cudaSuccess) e = launch_compress(p, qbar, kbar, vbar, ocg, idx, status_word, stream);
+    if (e == cudaSuccess) e = launch_compress(p, qbar, kbar, vbar, ocg, idx, status_word, nullptr, stream);
     if (e == cudaSuccess) e = launch_fine(p, q, k, v, gates, ocg, idx, out, status_word, stream);
     return from_cuda(e);
 }

@@ -35,8 +35,12 @@ cudaError_t launch_compress_select(const Problem &p, const float *qbar, const fl
                                    cudaStream_t stream);
 // tcgen05 three-pass tf32 path for (head_dim 64, top_n 16). Returns
 // cudaErrorNotSupported when it cannot take the problem. status: nullable.
+// images: nullable device scratch of compress_tc_workspace_bytes(p) bytes
+// (16-byte aligned); with it the tf32 split is done once per slab.
+bool compress_tc_supported(const Problem &p);
+size_t compress_tc_workspace_bytes(const Problem &p);
 cudaError_t launch_compress_tc(const Problem &p, const float *qbar, const float *kbar, const float *vbar,
-                               float *o_cg, int32_t *idx, uint32_t *status, cudaStream_t stream);
+                               float *o_cg, int32_t *idx, uint32_t *status, void *images, cudaStream_t stream);
 cudaError_t launch_attend_simt(const Problem &p, const void *q, const void *k, const void *v,
                                const float *gates, const float *o_cg, const int32_t *idx,
                                void *out, uint32_t *status, cudaStream_t stream);

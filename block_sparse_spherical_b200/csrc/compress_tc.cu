@@ -32,10 +32,15 @@
 // The row threads hold the tile's logits, their output row and their top-n
 // list in registers; a register split (setmaxnreg) moves registers to them
 // from the other warps, by whole warpgroups.
+// Given a workspace, a split kernel first writes every tile's tf32 parts, as
+// the byte image of its shared-memory layout, once per slab; the converter
+// warps then give way to one copy thread (bulk copies of those images), and no
+// CTA re-splits the slab's key tiles.
 // Every wait on an mbarrier is bounded (2 s); on expiry the CTA records a
 // timeout (when given a status word), writes -1 as its rows' block indices,
 // drains its MMAs and returns.
 #include <math_constants.h>
+#include <stddef.h>
 
 #include "tc_common.cuh"
 
@@ -75,9 +80,15 @@ struct alignas(1024) Smem {
 };
 
 static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory of one CTA");
+// Split images (per slab): Q row tile rt at rt·QIMG (hi regions, then lo), key
+// tile j of K and of V at j·KIMG (hi regions, then lo) in their own arrays.
+constexpr int QIMG = 4 * RROWS, KIMG = 4 * KROWS;
+static_assert(offsetof(Smem, qlo) == offsetof(Smem, qhi) + 2 * RROWS && offsetof(Smem, vlo) == offsetof(Smem, vhi) + 2 * KROWS,
+              "hi and lo parts adjacent, as in the split images");
 
 struct Args {
     const float *q, *k, *v;                // this slab's q̄, k̄, v̄ [m][64]
+    const uint8_t *qimg, *kimg, *vimg;     // this slab's split images (workspace path), else null
     float *o_cg;                           // this slab's [m][64]
     int32_t *idx;                          // this slab's [m][n]
     int m;
@@ -175,6 +186,56 @@ __device__ void convert_role(const Args &a, Smem &sh, int t, int row0, int T, vo
         convert_v(a.v, j * BN, a.m, t, sh.vhi[0], sh.vhi[1], sh.vlo[0], sh.vlo[1]);
         fence_proxy_async();
         mbar_arrive(&sh.v_full);
+    }
+}
+
+// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) completing on `bar`.
+__device__ __forceinline__ void bulk_copy(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Workspace path: one thread copies the split images in the converters'
+// order (Q; K(0); per tile j, K(j+1) and V(j)).
+__device__ void copy_role(const Args &a, Smem &sh, int row0, int T, volatile int *abort_flag) {
+    // most recent copy of each kind (for the drain on abort): K stage and parity, V parity
+    bool q_issued = false;
+    int last_kst = -1, last_vpar = -1;
+    uint32_t last_kpar = 0;
+    auto wait_c = [&](uint64_t *b, uint32_t par) -> bool {
+        return mbar_try_wait(b, par) || wait_bar(b, par, abort_flag, a.status);
+    };
+    auto copy_k = [&](int x) -> bool {      // K(x) into stage x%2 once S(x-2) has read it
+        const int st = x & 1;
+        if (!wait_c(&sh.k_empty[st], ((x >> 1) & 1) ^ 1)) return false;
+        mbar_expect_tx(&sh.k_full[st], KIMG);
+        bulk_copy(sh.khi[st][0], a.kimg + (int64_t)x * KIMG, 2 * KROWS, &sh.k_full[st]);
+        bulk_copy(sh.klo[st][0], a.kimg + (int64_t)x * KIMG + 2 * KROWS, 2 * KROWS, &sh.k_full[st]);
+        last_kst = st;
+        last_kpar = (x >> 1) & 1;
+        return true;
+    };
+    bool ok = true;
+    mbar_expect_tx(&sh.q_full, QIMG);
+    bulk_copy(sh.qhi[0], a.qimg + (int64_t)(row0 / BM) * QIMG, QIMG, &sh.q_full);
+    q_issued = true;
+    ok = copy_k(0);
+    for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T && !(ok = copy_k(j + 1))) break;
+        if (!(ok = wait_c(&sh.v_empty, (j & 1) ^ 1))) break;
+        mbar_expect_tx(&sh.v_full, KIMG);
+        bulk_copy(sh.vhi[0], a.vimg + (int64_t)j * KIMG, KIMG, &sh.v_full);
+        last_vpar = j & 1;
+    }
+    if (!ok) {                              // let the copies in flight land before the CTA exits
+        if (q_issued) drain_bar(&sh.q_full, 0);
+        if (last_kst >= 0) {
+            drain_bar(&sh.k_full[last_kst], last_kpar);
+            drain_bar(&sh.k_full[last_kst ^ 1], last_kpar ^ (last_kst == 0 ? 1u : 0u));
+        }
+        if (last_vpar >= 0) drain_bar(&sh.v_full, (uint32_t)last_vpar);
     }
 }
 
@@ -421,10 +482,11 @@ __device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter
     for (int p = 0; p < NSEL / 4; ++p) idst[p] = make_int4(li[4 * p], li[4 * p + 1], li[4 * p + 2], li[4 * p + 3]);
 }
 
-template <int NSEL>
+template <int NSEL, bool PRE>
 __global__ void __launch_bounds__(NTHREADS, 1)
 compress_tc_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar, const float *__restrict__ vbar,
-                   float *__restrict__ o_cg, int32_t *__restrict__ idx, int m, float sl2, uint32_t *status) {
+                   float *__restrict__ o_cg, int32_t *__restrict__ idx, int m, float sl2, uint32_t *status,
+                   const uint8_t *__restrict__ images) {
     extern __shared__ uint8_t smem_raw[];
     Smem &sh = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -440,18 +502,26 @@ compress_tc_kernel(const float *__restrict__ qbar, const float *__restrict__ kba
     a.m = m;
     a.sl2 = sl2;
     a.status = status;
+    a.qimg = a.kimg = a.vimg = nullptr;
+    if (PRE) {
+        const int64_t qbytes = (int64_t)((m + BM - 1) / BM) * QIMG, kbytes = (int64_t)T * KIMG;
+        a.qimg = images + slab * (qbytes + 2 * kbytes);
+        a.kimg = a.qimg + qbytes;
+        a.vimg = a.kimg + kbytes;
+    }
     volatile int *abort_flag = &sh.abort_flag;
+    constexpr uint32_t kFill = PRE ? 1u : 128u;   // arrivals that complete a Q/K/V tile
 
     if (threadIdx.x == 0) {
         sh.abort_flag = 0;
-        mbar_init(&sh.q_full, 128);
-        mbar_init(&sh.v_full, 128);
+        mbar_init(&sh.q_full, kFill);
+        mbar_init(&sh.v_full, kFill);
         mbar_init(&sh.v_empty, 1);
         mbar_init(&sh.p_full, 128);
         mbar_init(&sh.p_empty, 1);
         mbar_init(&sh.drain, 1);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sh.k_full[b], 128);
+            mbar_init(&sh.k_full[b], kFill);
             mbar_init(&sh.k_empty[b], 1);
             mbar_init(&sh.s_full[b], 1);
             mbar_init(&sh.s_free[b], 128);
@@ -477,9 +547,12 @@ compress_tc_kernel(const float *__restrict__ qbar, const float *__restrict__ kba
         softmax_role<NSEL>(a, sh, tmem, warp, lane, row0, T, abort_flag);
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
-        if (warp < 8)
+        if (PRE) {
+            if (warp == 4 && lane == 0) copy_role(a, sh, row0, T, abort_flag);
+        } else if (warp < 8) {
             convert_role(a, sh, threadIdx.x - 128, row0, T, abort_flag);
-        else if (warp == 8)
+        }
+        if (warp == 8)
             mma_role(a, sh, tmem, T, abort_flag);
     }
     __syncwarp();
@@ -493,25 +566,102 @@ compress_tc_kernel(const float *__restrict__ qbar, const float *__restrict__ kba
     }
 }
 
-}  // namespace
+// The split images of one slab: CTA (c, slab) handles block rows 64c..64c+63
+// (zero past m): their Q rows, and, if they form a key tile, that tile's K
+// and transposed V (same layouts as the converters write to shared memory).
+__global__ void __launch_bounds__(256)
+split_images_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar, const float *__restrict__ vbar,
+                    uint8_t *__restrict__ images, int m) {
+    const int64_t slab = blockIdx.y;
+    const int r0 = blockIdx.x * 64, t = threadIdx.x;
+    const int T = (m + BN - 1) / BN;
+    const int64_t qbytes = (int64_t)((m + BM - 1) / BM) * QIMG, kbytes = (int64_t)T * KIMG;
+    uint8_t *qimg = images + slab * (qbytes + 2 * kbytes);
+    uint8_t *kimg = qimg + qbytes, *vimg = kimg + kbytes;
+    const float *q = qbar + slab * (int64_t)m * D, *k = kbar + slab * (int64_t)m * D, *v = vbar + slab * (int64_t)m * D;
+    // Q: rows r0.. are rows (r0 % 128).. of row tile r0 / 128
+    {
+        uint8_t *base = qimg + (int64_t)(r0 / BM) * QIMG + (r0 % BM) * 128;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = t + 256 * u, r = i >> 4, c4 = i & 15;
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r0 + r < m) x = __ldg(reinterpret_cast<const float4 *>(q + (int64_t)(r0 + r) * D) + c4);
+            const int reg = c4 >> 3;
+            store_split(base + reg * RROWS, base + 2 * RROWS + reg * RROWS, sw128_offset(r, c4 & 7), x);
+        }
+    }
+    if (r0 >= T * BN) return;
+    const int kt = r0 / BN;
+    {
+        uint8_t *base = kimg + (int64_t)kt * KIMG;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = t + 256 * u, r = i >> 4, c4 = i & 15;
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r0 + r < m) x = __ldg(reinterpret_cast<const float4 *>(k + (int64_t)(r0 + r) * D) + c4);
+            const int reg = c4 >> 3;
+            store_split(base + reg * KROWS, base + 2 * KROWS + reg * KROWS, sw128_offset(r, c4 & 7), x);
+        }
+    }
+    {
+        uint8_t *base = vimg + (int64_t)kt * KIMG;
+        const int kg = t & 15, fg = t >> 4;    // one 4x4 block per thread
+        float4 x[4];
+#pragma unroll
+        for (int a2 = 0; a2 < 4; ++a2) {
+            const int key = r0 + 4 * kg + a2;
+            x[a2] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (key < m) x[a2] = __ldg(reinterpret_cast<const float4 *>(v + (int64_t)key * D) + fg);
+        }
+        uint8_t *hi = base + (kg >> 3) * KROWS, *lo = base + 2 * KROWS + (kg >> 3) * KROWS;
+        store_split(hi, lo, sw128_offset(4 * fg + 0, kg & 7), make_float4(x[0].x, x[1].x, x[2].x, x[3].x));
+        store_split(hi, lo, sw128_offset(4 * fg + 1, kg & 7), make_float4(x[0].y, x[1].y, x[2].y, x[3].y));
+        store_split(hi, lo, sw128_offset(4 * fg + 2, kg & 7), make_float4(x[0].z, x[1].z, x[2].z, x[3].z));
+        store_split(hi, lo, sw128_offset(4 * fg + 3, kg & 7), make_float4(x[0].w, x[1].w, x[2].w, x[3].w));
+    }
+}
 
-cudaError_t launch_compress_tc(const Problem &p, const float *qbar, const float *kbar, const float *vbar,
-                               float *o_cg, int32_t *idx, uint32_t *status, cudaStream_t stream) {
-    if (p.head_dim != D || p.top_n != 16) return cudaErrorNotSupported;
-    if (p.m > 0x7fffffffLL / D) return cudaErrorNotSupported;
+template <bool PRE>
+cudaError_t launch_tc(const Problem &p, const float *qbar, const float *kbar, const float *vbar, float *o_cg,
+                      int32_t *idx, uint32_t *status, const uint8_t *images, cudaStream_t stream) {
     const size_t smem = sizeof(Smem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(compress_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(compress_tc_kernel<16, PRE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     // the register split must fit the registers the CTA is launched with
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, compress_tc_kernel<16>);
+    e = cudaFuncGetAttributes(&fa, compress_tc_kernel<16, PRE>);
     if (e != cudaSuccess) return e;
     if ((int64_t)fa.numRegs * NTHREADS < kRegsNeeded || fa.maxThreadsPerBlock < NTHREADS)
         return cudaErrorInvalidConfiguration;
     const dim3 grid((unsigned)((p.m + BM - 1) / BM), (unsigned)p.slabs);
-    compress_tc_kernel<16><<<grid, NTHREADS, smem, stream>>>(qbar, kbar, vbar, o_cg, idx, (int)p.m,
-                                                               p.scale * 1.4426950408889634f, status);
+    compress_tc_kernel<16, PRE><<<grid, NTHREADS, smem, stream>>>(qbar, kbar, vbar, o_cg, idx, (int)p.m,
+                                                                   p.scale * 1.4426950408889634f, status, images);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+bool compress_tc_supported(const Problem &p) {
+    return p.head_dim == D && p.top_n == 16 && p.m <= 0x7fffffffLL / D;
+}
+
+size_t compress_tc_workspace_bytes(const Problem &p) {
+    if (!compress_tc_supported(p)) return 0;
+    const size_t rt = (size_t)((p.m + BM - 1) / BM), kt = (size_t)((p.m + BN - 1) / BN);
+    return (size_t)p.slabs * (rt * QIMG + 2 * kt * KIMG);
+}
+
+cudaError_t launch_compress_tc(const Problem &p, const float *qbar, const float *kbar, const float *vbar,
+                               float *o_cg, int32_t *idx, uint32_t *status, void *images, cudaStream_t stream) {
+    if (!compress_tc_supported(p)) return cudaErrorNotSupported;
+    if (!images) return launch_tc<false>(p, qbar, kbar, vbar, o_cg, idx, status, nullptr, stream);
+    const dim3 sgrid((unsigned)((p.m + BM - 1) / BM * 2), (unsigned)p.slabs);
+    split_images_kernel<<<sgrid, 256, 0, stream>>>(qbar, kbar, vbar, static_cast<uint8_t *>(images), (int)p.m);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_tc<true>(p, qbar, kbar, vbar, o_cg, idx, status, static_cast<const uint8_t *>(images), stream);
 }
 
 }  // namespace bsa

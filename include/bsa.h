@@ -103,6 +103,19 @@ BSA_API bsa_status bsa_compress_select(const bsa_config *cfg, const float *qbar,
                                cudaStream_t stream);
 
 /*
+ * The same computation with a caller-owned device workspace (the one
+ * bsa_forward takes: >= bsa_workspace_size bytes, 256-byte aligned). On the
+ * tensor-core path it first writes the tf32 split of q̄, k̄, v̄ into the
+ * workspace once per slab, so that the compressed kernel need not split every
+ * key tile again in every CTA; results are identical to bsa_compress_select.
+ * Only the split region of the workspace is written (it is the region after
+ * the block indices); BSA_ERR_WORKSPACE if the workspace is missing or small.
+ */
+BSA_API bsa_status bsa_compress_select_ws(const bsa_config *cfg, const float *qbar, const float *kbar,
+                                  const float *vbar, float *o_cg_block, int32_t *sel_idx, void *workspace,
+                                  size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Branches (b) and (c) and the gated combine of the BSA section, given the
  * block-level compressed output and the selected block indices:
  *   out_t = g_CG,t·o_cg_block[i(t)] + g_FG,t·o_FG,t + g_L,t·o_L,t
@@ -115,8 +128,9 @@ BSA_API bsa_status bsa_fine_attention(const bsa_config *cfg, const void *q, cons
                               const float *gates, const float *o_cg_block, const int32_t *sel_idx,
                               void *out, uint32_t *status_word, cudaStream_t stream);
 
-/* Bytes of device workspace bsa_forward needs for cfg (pooled tensors, o_cg_block,
- * block indices and the status word). */
+/* Bytes of device workspace bsa_forward needs for cfg (status word, pooled
+ * tensors, o_cg_block, block indices, and, on the tensor-core compressed path,
+ * the tf32 split of the pooled tensors). */
 BSA_API bsa_status bsa_workspace_size(const bsa_config *cfg, size_t *bytes);
 
 /*

@@ -76,7 +76,12 @@ def test_workspace_size_layout(lib):
         pooled = cfg.slabs * cfg.n_blocks * cfg.head_dim * 4
         idx = cfg.slabs * cfg.n_blocks * cfg.top_n * 4
         up = lambda x: (x + 255) // 256 * 256
-        assert n == 256 + 4 * up(pooled) + up(idx)
+        split = 0
+        if cfg.head_dim == 64 and cfg.top_n == 16:   # tensor-core compressed path: tf32 split images
+            m = cfg.n_blocks
+            row_tiles, key_tiles = (m + 127) // 128, (m + 63) // 64
+            split = cfg.slabs * (row_tiles * 65536 + 2 * key_tiles * 32768)
+        assert n == 256 + 4 * up(pooled) + up(idx) + up(split)
 
 
 def test_null_and_misaligned_pointers_rejected_before_launch(lib):
@@ -97,8 +102,11 @@ def test_null_and_misaligned_pointers_rejected_before_launch(lib):
     assert L.bsa_forward(cp, A, A, A, A, A, None, A + 16, 1 << 30, None) == 3
     # workspace missing / too small
     assert L.bsa_forward(cp, A, A, A, A, A, None, None, 1 << 30, None) == 6
+    assert L.bsa_compress_select_ws(cp, A, A, A, A, A, None, 1 << 30, None) == 6
     _, need = ws_size(c)
     assert L.bsa_forward(cp, A, A, A, A, A, None, A, need - 1, None) == 6
+    assert L.bsa_compress_select_ws(cp, A, A, A, A, A, A, need - 1, None) == 6
+    assert L.bsa_compress_select_ws(cp, A, A, A, A, A, A + 16, need, None) == 3
     # bad config with good pointers
     bad = cfg_of(top_n=0)
     assert L.bsa_forward(ctypes.byref(bad), A, A, A, A, A, None, A, need, None) == 1

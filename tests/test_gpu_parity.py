@@ -167,3 +167,23 @@ def test_value_magnitude_range(log2_scale):
         b, h = divmod(s, cfg.heads)
         gpu = {"idx": parity.to_np(bsa.sel_idx[b, h]), "out": back[b, h].cpu().numpy()}
         parity.check_slab(cfg, s, gpu, None)
+
+
+@pytest.mark.parametrize("name", ["nside32", "tc_compress_m257"])
+def test_compress_with_workspace_matches(name):
+    """bsa_compress_select_ws (tf32 split once per slab into the workspace) gives bit-identical block
+    indices and compressed outputs to bsa_compress_select (split inside every CTA)."""
+    cfg = CONFIGS["nside32"]
+    if name != "nside32":
+        cfg = cfg.with_(name=name, tokens=64 * 257, heads=3, window_blocks=2, seed=7)
+    q, k, v, g = parity.device_inputs(cfg)
+    qb, kb, vb = api.pool(q, k, v, cfg.block_size)
+    o1, i1 = api.compress_select(qb, kb, vb, cfg.top_n, cfg.block_size)
+    c = abi.make_config(cfg)
+    nbytes = abi.bsa_workspace_size(c)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    o2, i2 = torch.empty_like(o1), torch.empty_like(i1)
+    abi.bsa_compress_select_ws(c, qb, kb, vb, o2, i2, ws, nbytes)
+    torch.cuda.synchronize()
+    assert torch.equal(i1, i2)
+    assert torch.equal(o1, o2)
