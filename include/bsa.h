@@ -34,7 +34,9 @@
  *      {(BSA_F32, 16, 32), (BSA_F32, 64, 64), (BSA_BF16, 64, 64)}
  *    with 1 <= top_n <= min(m, 64) and window_blocks >= 0. bf16 inputs use
  *    bf16 tensor-core products with fp32 accumulation; the compressed
- *    branch and the top-n decision are computed in fp32.
+ *    branch and the top-n decision are fp32-accurate (fp32 on the CUDA
+ *    cores, or, for head_dim 64 and top_n 16, three-pass tf32 products on
+ *    the tensor cores).
  */
 #ifndef BSA_H
 #define BSA_H
