@@ -228,9 +228,10 @@ const char *bsa_status_string(bsa_status s) {
 // that executes inside a host callback or another library's allocator hook,
 // plugins whose host framework owns every device allocation, or services
 // that must not touch the allocator on the request path. For them,
-// bsa_forward_noalloc runs the same three kernels as bsa_forward but keeps
-// the intermediates (pooled q̄/k̄/v̄, block-level compressed output, block
-// indices) in a fixed array of device memory that this library owns.
+// bsa_forward_noalloc computes what bsa_forward computes but keeps the
+// intermediates (pooled q̄/k̄/v̄, block-level compressed output, block
+// indices) in a fixed array of device memory that this library owns; its
+// compressed branch splits operands in every CTA (no space for split images).
 //
 // The array lives in device global memory for as long as the library is
 // loaded, on every GPU that loads it, and is shared by every call on that

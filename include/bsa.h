@@ -162,13 +162,17 @@ BSA_API bsa_status bsa_check_status(const void *status_word, cudaStream_t stream
  * For callers that cannot allocate device memory when they run BSA (code in
  * a host callback or an allocator hook, plugins whose host framework owns all
  * device allocations, request paths that must not touch the allocator). It
- * runs the same three kernels as bsa_forward, but the intermediates live in
- * a fixed 32 MiB array of device memory owned by the library instead of a
- * caller workspace; the caller still passes q, k, v, gates and out (and the
+ * computes what bsa_forward computes (bit for bit), but the intermediates
+ * live in a fixed 32 MiB array of device memory owned by the library instead
+ * of a caller workspace, and the compressed branch splits its operands inside
+ * every CTA, as bsa_compress_select does; the caller still passes q, k, v,
+ * gates and out (and the
  * optional sel_idx_out / status_word, same meaning as in bsa_forward and
  * bsa_fine_attention; status_word may be NULL).
- *  - Returns BSA_ERR_WORKSPACE when bsa_workspace_size(cfg) exceeds 32 MiB
- *    (e.g. Nside 64 with batch 4 x 8 heads fits; Nside 128 with 2 x 16 does not).
+ *  - Returns BSA_ERR_WORKSPACE when the intermediates (status word, pooled
+ *    tensors, o_cg_block, block indices: bsa_workspace_size without the
+ *    compressed kernel's split images) exceed 32 MiB (e.g. Nside 64 with
+ *    batch 4 x 8 heads fits; Nside 128 with 2 x 16 does not).
  *  - Never calls cudaMalloc, cudaFree or any allocating routine.
  *  - The array exists on every GPU that loads the library until the process
  *    exits. The first call on each device looks up its device address (with
