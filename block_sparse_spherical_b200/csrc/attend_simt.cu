@@ -136,8 +136,7 @@ cudaError_t launch(const Problem &p, const void *q, const void *k, const void *v
 cudaError_t launch_attend_simt(const Problem &p, const void *q, const void *k, const void *v,
                                const float *gates, const float *o_cg, const int32_t *idx,
                                void *out, uint32_t *status, cudaStream_t stream) {
-    if (p.dtype == BSA_BF16 && p.block_size == 64 && p.head_dim == 64)
-        return launch<__nv_bfloat16, 64, 64>(p, q, k, v, gates, o_cg, idx, out, status, stream);
+    // fp32 workloads only: bf16 fine attention runs on the tensor cores and nowhere else
     if (p.dtype == BSA_F32 && p.block_size == 64 && p.head_dim == 64)
         return launch<float, 64, 64>(p, q, k, v, gates, o_cg, idx, out, status, stream);
     if (p.dtype == BSA_F32 && p.block_size == 16 && p.head_dim == 32)

@@ -626,7 +626,7 @@ cudaError_t launch_attend_tc(const Problem &pb, const void *q, const void *k, co
     if (rows > 0x7fffffffLL) return cudaErrorNotSupported;       // TMA row coordinate is int32
     CUtensorMap tq, tk, tv;
     if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows))
-        return cudaErrorNotSupported;
+        return cudaErrorInvalidValue;        // driver entry point missing or tensor map rejected
     TcParams p;
     p.idx = idx;
     p.gates = gates;
@@ -641,7 +641,7 @@ cudaError_t launch_attend_tc(const Problem &pb, const void *q, const void *k, co
     p.scale_log2 = pb.scale * 1.4426950408889634f;
     p.withhold_v_step = pb.withhold_v_step;
     const int sms = sm_count();
-    if (sms <= 0) return cudaErrorNotSupported;
+    if (sms <= 0) return cudaErrorInvalidDevice;
     const int64_t want = (p.total_blocks + NSLOT - 1) / NSLOT;
     const int grid = (int)(want < sms ? want : sms);
     const size_t smem = sizeof(SharedStorage) + 1024;

@@ -34,6 +34,8 @@ bsa_status make_problem(const bsa_config *cfg, Problem *p) {
     if (cfg->top_n > bsa::kMaxTopN) return BSA_ERR_UNSUPPORTED;
     const int64_t slabs = (int64_t)cfg->batch * cfg->heads;
     if (slabs > 65535) return BSA_ERR_UNSUPPORTED;            // grid.y of the per-slab kernels
+    // the tensor-core kernel addresses token rows with 32-bit TMA coordinates
+    if (cfg->dtype == BSA_BF16 && slabs * cfg->n_tokens > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
     p->batch = cfg->batch;
     p->heads = cfg->heads;
     p->n_tokens = cfg->n_tokens;
@@ -86,11 +88,12 @@ cudaError_t launch_compress(const Problem &p, const float *qbar, const float *kb
     return bsa::launch_compress_select(p, qbar, kbar, vbar, o_cg, idx, stream);
 }
 
+// Selection + local branches and the combine: bf16 problems run on the tensor cores only (a
+// failure there is returned, never retried elsewhere); fp32 problems on the CUDA cores.
 cudaError_t launch_fine(const Problem &p, const void *q, const void *k, const void *v,
                         const float *gates, const float *o_cg, const int32_t *idx, void *out,
                         uint32_t *status, cudaStream_t stream) {
-    cudaError_t e = bsa::launch_attend_tc(p, q, k, v, gates, o_cg, idx, out, status, stream);
-    if (e != cudaErrorNotSupported) return e;
+    if (p.dtype == BSA_BF16) return bsa::launch_attend_tc(p, q, k, v, gates, o_cg, idx, out, status, stream);
     return bsa::launch_attend_simt(p, q, k, v, gates, o_cg, idx, out, status, stream);
 }
 
@@ -241,6 +244,8 @@ const char *bsa_status_string(bsa_status s) {
 // previous call are never used.
 // ---------------------------------------------------------------------------
 
+#include <cuda.h>
+
 #include <mutex>
 
 namespace {
@@ -252,26 +257,72 @@ static __device__ __align__(256) unsigned char g_bsa_noalloc_scratch[kNoAllocScr
 
 namespace {
 
-std::once_flag g_scratch_once[kMaxDevices];
-void *g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+// The scratch array's device address is a property of the CUDA context that
+// loaded this library's module: a new primary context (after cudaDeviceReset,
+// for instance) loads the module again, and the array may then sit elsewhere.
+// So the address is cached per device together with the id of the context it
+// was looked up in (cuCtxGetId: unique for the life of the process, never
+// reused), and looked up again, with that device current, whenever the
+// current context is another one. Failed lookups are not cached.
+struct ScratchSlot {
+    std::mutex mu;
+    unsigned long long ctx_id = 0;   // 0: nothing cached
+    void *ptr = nullptr;
+};
+ScratchSlot g_scratch[kMaxDevices];
 
-// Device address of the scratch array on the current device. In host code
-// the array's name only stands in for it, so the address is looked up once
-// per device, with that device current, on the first call made there.
+typedef CUresult (*PFN_ctx_get_current)(CUcontext *);
+typedef CUresult (*PFN_ctx_get_id)(CUcontext, unsigned long long *);
+
+bool driver_fn(const char *name, void **fn) {
+    cudaDriverEntryPointQueryResult q;
+    return cudaGetDriverEntryPoint(name, fn, cudaEnableDefault, &q) == cudaSuccess &&
+           q == cudaDriverEntryPointSuccess && *fn != nullptr;
+}
+
+// Id of the calling thread's current context, or 0 if there is none (yet).
+cudaError_t current_ctx_id(unsigned long long *id) {
+    static PFN_ctx_get_current get_current = nullptr;
+    static PFN_ctx_get_id get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        if (driver_fn("cuCtxGetCurrent", &f)) get_current = reinterpret_cast<PFN_ctx_get_current>(f);
+        f = nullptr;
+        if (driver_fn("cuCtxGetId", &f)) get_id = reinterpret_cast<PFN_ctx_get_id>(f);
+    });
+    if (!get_current || !get_id) return cudaErrorNotSupported;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    *id = 0;
+    if (ctx && get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    return cudaSuccess;
+}
+
+// Device address of the scratch array in the current device's current context.
+// In host code the array's name only stands in for it, so the address is
+// looked up with cudaGetSymbolAddress, once per device and context, on the
+// first call made there.
 cudaError_t noalloc_scratch(void **out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::call_once(g_scratch_once[dev], [dev] {
-        void *p = nullptr;
-        g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_bsa_noalloc_scratch);
-        g_scratch_ptr[dev] = p;
-    });
-    if (g_scratch_err[dev] != cudaSuccess) return g_scratch_err[dev];
-    if (!g_scratch_ptr[dev]) return cudaErrorInvalidSymbol;
-    *out = g_scratch_ptr[dev];
+    ScratchSlot &slot = g_scratch[dev];
+    std::lock_guard<std::mutex> lock(slot.mu);
+    unsigned long long id = 0;
+    if ((e = current_ctx_id(&id)) != cudaSuccess) return e;
+    if (id != 0 && id == slot.ctx_id && slot.ptr) {
+        *out = slot.ptr;
+        return cudaSuccess;
+    }
+    void *p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_bsa_noalloc_scratch)) != cudaSuccess) return e;   // not cached
+    if (!p) return cudaErrorInvalidSymbol;
+    if ((e = current_ctx_id(&id)) != cudaSuccess) return e;   // the lookup may have created the context
+    slot.ctx_id = id;
+    slot.ptr = p;
+    *out = p;
     return cudaSuccess;
 }
 

@@ -44,8 +44,8 @@ cudaError_t launch_compress_tc(const Problem &p, const float *qbar, const float 
 cudaError_t launch_attend_simt(const Problem &p, const void *q, const void *k, const void *v,
                                const float *gates, const float *o_cg, const int32_t *idx,
                                void *out, uint32_t *status, cudaStream_t stream);
-// tcgen05/TMA path for (bf16, block 64, d 64). Returns cudaErrorNotSupported
-// when it cannot take the problem, so that the caller can pick another kernel.
+// tcgen05/TMA path for (bf16, block 64, d 64), the only kernel for bf16 fine
+// attention. Returns cudaErrorNotSupported for shapes it does not take.
 cudaError_t launch_attend_tc(const Problem &p, const void *q, const void *k, const void *v,
                              const float *gates, const float *o_cg, const int32_t *idx,
                              void *out, uint32_t *status, cudaStream_t stream);

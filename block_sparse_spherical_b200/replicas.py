@@ -52,5 +52,11 @@ def barrier(device=None) -> None:
 
 
 def job_tokens_per_step(cfg: BSAConfig, world: int) -> int:
-    """Tokens processed by all ranks in one step (each rank runs a full batch)."""
+    """Tokens (batch x N; every head of a token counted once) processed by all ranks in one step
+    (each rank runs a full batch)."""
+    return world * cfg.batch * cfg.n_tokens
+
+
+def job_head_rows_per_step(cfg: BSAConfig, world: int) -> int:
+    """Query rows (batch x heads x N) processed by all ranks in one step."""
     return world * cfg.slabs * cfg.n_tokens

@@ -177,6 +177,9 @@ BSA_API bsa_status bsa_check_status(const void *status_word, cudaStream_t stream
  *  - The array exists on every GPU that loads the library until the process
  *    exits. The first call on each device looks up its device address (with
  *    that device current); make that first call before any stream capture.
+ *    The address is remembered per device and CUDA context: a call made in a
+ *    new context of the device (e.g. after cudaDeviceReset) looks it up
+ *    again, and a lookup that fails is retried by the next call.
  *  - All calls on a GPU share the array: calls that overlap on the GPU
  *    (other streams, other host threads) race and must be serialised by the
  *    caller. Each call rewrites everything it reads, so no part of the array

@@ -48,6 +48,11 @@ def load(path: str | None = None):
     return lib
 
 
+def load_native():
+    """The oracle built with -O3 -march=native on this host (same results; for CPU timings)."""
+    return load(_build.build_native())
+
+
 def _f64(x) -> np.ndarray:
     return np.ascontiguousarray(x, dtype=np.float64)
 
@@ -144,4 +149,4 @@ def forward_slab(q, k, v, gates, block: int, n: int, w: int, scale: float | None
     return {"out": out, "qbar": qb, "kbar": kb, "vbar": vb, "o_cg": ocg, "idx": idx, "gap": gap}
 
 
-__all__ = ["load", "pool", "compressed_rows", "fine_rows", "forward_slab", "default_scale"]
+__all__ = ["load", "load_native", "pool", "compressed_rows", "fine_rows", "forward_slab", "default_scale"]

@@ -113,6 +113,20 @@ def test_null_and_misaligned_pointers_rejected_before_launch(lib):
     assert L.bsa_pool(None, A, A, A, A, A, A, None) == 1
 
 
+def test_bf16_shape_beyond_the_tensor_core_kernel_is_an_error(lib):
+    """bf16 fine attention runs on the tensor-core kernel only: a bf16 problem that kernel cannot
+    address (more than 2^31 - 1 token rows for its 32-bit TMA coordinates) is refused with
+    BSA_ERR_UNSUPPORTED on the host, never sent to another kernel."""
+    L = abi.load()
+    A = 4096          # never dereferenced: validation fails first
+    big = cfg_of(batch=1, heads=2, n_tokens=1 << 30)
+    assert L.bsa_fine_attention(ctypes.byref(big), A, A, A, A, A, A, A, None, None) == 2
+    assert L.bsa_forward(ctypes.byref(big), A, A, A, A, A, None, A, 1 << 62, None) == 2
+    assert ws_size(big)[0] == 2
+    # the same row count in fp32 is a valid problem for the CUDA-core kernels
+    assert ws_size(cfg_of(batch=1, heads=2, n_tokens=1 << 30, dtype=0))[0] == 0
+
+
 def test_python_binding_raises_on_error(lib):
     c = cfg_of(top_n=0)
     with pytest.raises(abi.BsaError) as e:

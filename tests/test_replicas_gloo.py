@@ -16,8 +16,8 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 from block_sparse_spherical_b200.configs import CONFIGS
-from block_sparse_spherical_b200.replicas import (barrier, job_tokens_per_step, max_over_ranks,
-                                                  replica_config)
+from block_sparse_spherical_b200.replicas import (barrier, job_head_rows_per_step, job_tokens_per_step,
+                                                  max_over_ranks, replica_config)
 
 
 def _free_port():
@@ -55,7 +55,7 @@ def test_two_gloo_replicas(tmp_path):
     assert not np.array_equal(r[0]["out"], r[1]["out"]), "replicas must run independent inputs"
     for x in r:
         assert float(x["worst"]) == 15.0          # max over ranks, seen by every rank
-        assert int(x["tokens"]) == 2 * CONFIGS["tiny_nside8"].slabs * CONFIGS["tiny_nside8"].n_tokens
+        assert int(x["tokens"]) == 2 * CONFIGS["tiny_nside8"].batch * CONFIGS["tiny_nside8"].n_tokens
 
 
 def test_single_process_helpers_without_a_process_group():
@@ -63,4 +63,5 @@ def test_single_process_helpers_without_a_process_group():
     barrier()
     cfg = CONFIGS["nside128"]
     assert replica_config(cfg, 0) is cfg
-    assert job_tokens_per_step(cfg, 8) == 8 * 2 * 16 * 196608
+    assert job_tokens_per_step(cfg, 8) == 8 * 2 * 196608
+    assert job_head_rows_per_step(cfg, 8) == 8 * 2 * 16 * 196608

@@ -4,9 +4,9 @@ bsa_forward_noalloc exists for callers that cannot allocate device memory
 when they run BSA (allocator hooks, host callbacks, plugins whose framework
 owns all device memory): it keeps its intermediates in a fixed scratch array
 owned by the library. This test calls it through the C ABI twice in a row and
-compares each result with bsa_forward (caller workspace) within the parity
-tolerances of the other GPU tests, and checks that a problem too large for
-the scratch is refused. It lives in its own file, collected last, and builds
+compares each result with bsa_forward (caller workspace): within the parity
+tolerances of the other GPU tests and, as its header promises, bit for bit;
+and it checks that a problem too large for the scratch is refused. It lives in its own file, collected last, and builds
 its own inputs, so it passes alone in a fresh process or after the rest.
 """
 import ctypes
@@ -47,6 +47,8 @@ def test_noalloc_matches_workspace_forward_twice(name):
         assert abi.bsa_check_status(status) == 0, f"call {call}: device status word set"
         assert torch.equal(idx, ref_bsa.sel_idx), f"call {call}: selected blocks differ"
         parity.check_output(parity.to_np(out), parity.to_np(ref), cfg.dtype, f"{name} no-alloc call {call}")
+        # the header promises the same result as bsa_forward bit for bit
+        assert torch.equal(out, ref), f"call {call}: output differs from bsa_forward"
 
 
 def test_noalloc_without_optional_outputs():
@@ -57,6 +59,7 @@ def test_noalloc_without_optional_outputs():
     abi.bsa_forward_noalloc(abi.make_config(cfg), q, k, v, g, out, None, None)
     torch.cuda.synchronize()
     parity.check_output(parity.to_np(out), parity.to_np(ref), cfg.dtype, "no-alloc without sel_idx/status")
+    assert torch.equal(out, ref)
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch():
