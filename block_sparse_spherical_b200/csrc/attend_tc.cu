@@ -59,24 +59,45 @@ constexpr int TILE = BK * HD * 2;           // bytes of one 64x64 bf16 tile
 #ifndef BSA_TC_STAGES
 #define BSA_TC_STAGES 2
 #endif
+#ifndef BSA_TC_P_TMEM
+#define BSA_TC_P_TMEM 1
+#endif
 constexpr int NSLOT = BSA_TC_SLOTS;        // independent pipelines per CTA
 constexpr int NSTAGE = BSA_TC_STAGES;      // depth of the K and V rings
+constexpr bool P_TMEM = BSA_TC_P_TMEM != 0;   // P·V reads P from tensor memory (else shared memory)
 constexpr int NTHREADS = 32 * (2 * NSLOT + 4 * NSLOT);
 // Register split (setmaxnreg): the two control warpgroups (MMA issuers, loaders)
 // drop to kCtrlRegs, the softmax warpgroups rise to kSoftRegs. The sum must not
 // exceed what the CTA was launched with; the host checks the compiled count.
 constexpr int kCtrlRegs = 48, kSoftRegs = 96;
 constexpr int kRegsNeeded = 2 * NSLOT * 32 * kCtrlRegs + 4 * NSLOT * 32 * kSoftRegs;
-constexpr uint32_t TMEM_COLS = 512;         // per slot: S and O, 64 columns each
+constexpr uint32_t TMEM_COLS = 512;         // 128 columns per slot
 constexpr float kRescaleLog2 = 8.0f;        // lazy rescale threshold (factor 256)
 
+// Tensor-memory map of a slot (128 columns). An M=64 accumulator occupies 16
+// of the 32 lanes of each sub-partition (row r in lane 32*(r/16) + r%16 + base,
+// base 0 or 16), so two of them can share columns in the two lane halves.
+//   O   (P·V accumulator)                       columns  0..63,  lanes +0
+//   S   (Q·Kᵀ scores)                           columns  0..63,  lanes +16   (P in TMEM)
+//                                               columns 64..127, lanes +0    (P in shared memory)
+//   P   (softmax numerators, bf16 pairs, the A  columns 64..95 / 96..127 (buffer 0 / 1),
+//        operand of P·V; two buffers)           lanes +0, same lanes as O as the MMA requires
+//   acc (fp32 g_CG·o_CG + g_FG·o_FG, written    columns 64..127, lanes +16
+//        and read only by the softmax threads)
+constexpr uint32_t O_COL = 0, O_LANE = 0;
+constexpr uint32_t S_COL = P_TMEM ? 0 : 64, S_LANE = P_TMEM ? 16 : 0;
+constexpr uint32_t P_COL = 64, P_LANE = 0;
+constexpr uint32_t ACC_COL = 64, ACC_LANE = 16;
+static_assert(P_TMEM || (S_COL != O_COL || S_LANE != O_LANE), "S and O overlap");
+
+constexpr int NPBUF_SMEM = P_TMEM ? 0 : 2;
 struct alignas(1024) SlotTiles {
     uint8_t q[TILE];
     uint8_t k[NSTAGE][TILE];   // [stage]
     uint8_t v[NSTAGE][TILE];   // [stage]
-    uint8_t p[2][TILE];        // [buffer]: P(g) in buffer g%2
+    uint8_t p[NPBUF_SMEM > 0 ? NPBUF_SMEM : 1][NPBUF_SMEM > 0 ? TILE : 1024];   // [buffer]: P(g) in buffer g%2
 };
-static_assert(sizeof(SlotTiles) == (3 + 2 * NSTAGE) * TILE, "tile layout");
+static_assert(sizeof(SlotTiles) == (1 + 2 * NSTAGE) * TILE + (P_TMEM ? 1024 : 2 * TILE), "tile layout");
 
 struct SlotBars {
     uint64_t q_full, q_empty;
@@ -119,6 +140,17 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
         : "memory");
 }
 
+// D (TMEM) (+)= A·B with A (K-major bf16 pairs, the lanes of D) read from tensor memory.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // 16 lanes x 16 columns twice: thread t of the warp gets TMEM lane (base + t%16),
 // columns [col, col+16) for t < 16 and [col+32, col+48) for t >= 16.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *r) {
@@ -129,6 +161,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *r) {
         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
           "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
         : "r"(taddr));
+}
+// 16 lanes x 16 columns: thread t < 16 writes lane (base + t) columns [col, col+16), thread
+// t >= 16 writes lane (base + t - 16) columns [col+16, col+32): one row's 32 bf16 pairs.
+__device__ __forceinline__ void tmem_st16_pairs(uint32_t taddr, const uint32_t *u) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 16, "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "r"(u[8]),
+        "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
+        : "memory");
 }
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *r) {
     const uint32_t *u = reinterpret_cast<const uint32_t *>(r);
@@ -267,11 +309,12 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
                          volatile int *abort_flag) {
     const int L = 2 * p.w + 1, T = L + p.n;
     const int64_t stride = NSLOT * (int64_t)gridDim.x;
-    const uint32_t tS = tmem_slot, tO = tmem_slot + 64;
+    const uint32_t tS = tmem_slot + S_COL + (S_LANE << 16), tO = tmem_slot + O_COL + (O_LANE << 16);
+    const uint32_t tP = tmem_slot + P_COL + (P_LANE << 16);   // P buffer b at + 32*b (P in TMEM)
     // shared-memory descriptors of every operand tile, computed once
     const uint64_t dq = desc_kmajor(S.q);
     const uint64_t dk0 = desc_kmajor(S.k[0]), dv0 = desc_mnmajor(S.v[0]);   // stage s: + s*TILE/16
-    const uint64_t dp0 = desc_kmajor(S.p[0]), dp1 = desc_kmajor(S.p[1]);
+    const uint64_t dp0 = desc_kmajor(S.p[0]), dp1 = desc_kmajor(S.p[NPBUF_SMEM > 1 ? 1 : 0]);
     uint32_t c = 0, g = 0;
     bool ok = true;
     const bool leader = elect_one();       // issues MMAs and commits; the whole warp runs the loop
@@ -311,8 +354,15 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
             const uint64_t dv = dv0 + (uint64_t)(vs * (TILE >> 4));
             const uint64_t dp = pb ? dp1 : dp0;
             if (leader) {
+                if (P_TMEM) {
+                    // K chunk kk (16 keys) of P = 8 columns of bf16 pairs
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) tc_mma(tO, dp + 2 * kk, dv + 128 * kk, kIdescPV, kk ? 1u : acc0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_ts(tO, tP + 32u * pb + 8u * kk, dv + 128 * kk, kIdescPV, kk ? 1u : acc0);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) tc_mma(tO, dp + 2 * kk, dv + 128 * kk, kIdescPV, kk ? 1u : acc0);
+                }
                 commit(&B.o_done[pb]);
                 commit(&B.v_empty[vs]);
                 commit(&B.p_empty[pb]);
@@ -334,8 +384,11 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
     const int L = 2 * p.w + 1, T = L + p.n;
     const int ch = lane >> 4;              // column half of the row
     const int r = 16 * wq + (lane & 15);   // row within the query block
-    const uint32_t tlane = (uint32_t)(32 * wq) << 16;
-    const uint32_t tS = tmem_slot + tlane, tO = tmem_slot + 64 + tlane;
+    const uint32_t wl = (uint32_t)(32 * wq);   // this warp's sub-partition
+    const uint32_t tS = tmem_slot + S_COL + ((wl + S_LANE) << 16);
+    const uint32_t tO = tmem_slot + O_COL + ((wl + O_LANE) << 16);
+    const uint32_t tA = tmem_slot + ACC_COL + ((wl + ACC_LANE) << 16);
+    const uint32_t tP = tmem_slot + P_COL + ((wl + P_LANE) << 16);
     const int prow_off = (r >> 3) * 1024 + (r & 7) * 128;
     const int sw = r & 7;
     const float sl2 = p.scale_log2;
@@ -377,8 +430,6 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 if (lane + 32 < p.n) j1 = __ldg(ix + lane + 32);
             }
         }
-        __half2 acc[16];                   // acc / acc_scale, fp16 pairs
-        float acc_scale = 1.f;
         float m_used = -INFINITY, l_run = 0.f, l_sel = 0.f;
         for (int t = 0; t < T; ++t, ++g) {
             bool valid;
@@ -435,28 +486,19 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             if (touch_o && g > 0 && !(ok = wait_all(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1))) break;
             fence_after();
             if (t == p.n) {
-                // close the selection branch: acc = g_CG·o_CG + g_FG·o_FG
+                // close the selection branch: acc = g_CG·o_CG + g_FG·o_FG, kept in fp32 in
+                // this row's lanes of the other lane half until the epilogue
                 const float l = l_sel + __shfl_xor_sync(FULL, l_sel, 16);
                 const float inv = l > 0.f ? g_fg / l : 0.f;
                 float a[32];
                 tmem_ld16(tO, a);
                 tmem_ld16(tO + 16, a + 16);
                 tmem_wait_ld();
-                float amax = 0.f;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    a[e] = fmaf(g_cg, __ldg(ocg + e), a[e] * inv);
-                    amax = fmaxf(amax, fabsf(a[e]));
-                }
-                // power-of-two scale 2^k that puts this thread's largest |acc| in
-                // [2^14, 2^15): the fp16 copy neither overflows nor goes subnormal
-                // (all-zero or non-finite values are stored unscaled)
-                const int ex = (__float_as_int(amax) >> 23) & 0xff;
-                const int k = (ex == 0 || ex == 255) ? 0 : min(max(ex - 141, -112), 113);
-                acc_scale = __int_as_float((127 + k) << 23);
-                const float down = __int_as_float((127 - k) << 23);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) acc[e] = __floats2half2_rn(a[2 * e] * down, a[2 * e + 1] * down);
+                for (int e = 0; e < 32; ++e) a[e] = fmaf(g_cg, __ldg(ocg + e), a[e] * inv);
+                tmem_st16(tA, a);
+                tmem_st16(tA + 16, a + 16);
+                tmem_wait_st();
             } else if (touch_o) {
                 // rows whose running max grew by more than 2^8: rescale their O and sum
                 const float alpha = need ? ex2(m_old - m_used) : 1.f;
@@ -477,14 +519,20 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             //      K-major 128-byte swizzle, once P·V(g-2) has released that buffer
             const int pb = g & 1;
             if (!(ok = wait_all(&B.p_empty[pb], ((g >> 1) & 1) ^ 1))) break;
-            uint8_t *prow = S.p[pb] + prow_off;
+            if (P_TMEM) {
+                // P (bf16 pairs) into this row's lanes of P buffer pb: the A operand of P·V
+                tmem_st16_pairs(tP + 32u * pb, pk);
+                tmem_wait_st();
+            } else {
+                uint8_t *prow = S.p[NPBUF_SMEM > 1 ? pb : 0] + prow_off;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const int chunk = 4 * ch + c4;
-                const uint4 v4 = make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
-                *reinterpret_cast<uint4 *>(prow + ((chunk ^ sw) << 4)) = v4;
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int chunk = 4 * ch + c4;
+                    const uint4 v4 = make_uint4(pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
+                    *reinterpret_cast<uint4 *>(prow + ((chunk ^ sw) << 4)) = v4;
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             fence_before();
             mbar_arrive(&B.p_full[pb]);        // every softmax thread arrives (count 128)
         }
@@ -497,15 +545,14 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
         uint4 *d4 = reinterpret_cast<uint4 *>(p.out + tok * HD + 32 * ch);
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-            float o[16];
+            float o[16], a[16];
             tmem_ld16(tO + 16 * cc, o);
+            tmem_ld16(tA + 16 * cc, a);
             tmem_wait_ld();
             uint32_t w8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float2 a2 = __half22float2(acc[8 * cc + e]);
-                w8[e] = pack_bf16(fmaf(o[2 * e], inv, a2.x * acc_scale), fmaf(o[2 * e + 1], inv, a2.y * acc_scale));
-            }
+            for (int e = 0; e < 8; ++e)
+                w8[e] = pack_bf16(fmaf(o[2 * e], inv, a[2 * e]), fmaf(o[2 * e + 1], inv, a[2 * e + 1]));
             d4[2 * cc] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
             d4[2 * cc + 1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
         }

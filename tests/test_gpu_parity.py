@@ -169,6 +169,31 @@ def test_value_magnitude_range(log2_scale):
         parity.check_slab(cfg, s, gpu, None)
 
 
+@pytest.mark.parametrize("spread", [2, 3])
+def test_value_channel_spread(spread):
+    """V's channels scaled by different exact powers of two, channel c by 2^(spread*(c mod 8)),
+    spanning 2^14 (spread 2) or 2^21 (spread 3). Selection does not depend on V and every output
+    channel is linear in its own V channel, so channel c of the output divided by its factor
+    must meet the bf16 tolerances against the oracle of the unscaled problem. This holds only if
+    the kernel carries each channel of the combined compressed + selection output at its own
+    precision (fp32), not under one scale shared by a thread's channels."""
+    cfg = CONFIGS["nside32"]
+    q, k, v, g = parity.device_inputs(cfg)
+    c = torch.arange(cfg.head_dim, device="cuda")
+    f = torch.pow(2.0, (spread * (c % 8)).double()).float()
+    vs = (v.float() * f).to(torch.bfloat16)
+    assert torch.equal(vs.float() / f, v.float())
+    bsa = api.BSA.from_config(cfg)
+    out = bsa(q, k, vs, g)
+    torch.cuda.synchronize()
+    assert bsa.check_status() == 0
+    back = (out.float() / f).to(torch.float64)
+    for s in range(cfg.slabs):
+        b, h = divmod(s, cfg.heads)
+        gpu = {"idx": parity.to_np(bsa.sel_idx[b, h]), "out": back[b, h].cpu().numpy()}
+        parity.check_slab(cfg, s, gpu, None)
+
+
 @pytest.mark.parametrize("name", ["nside32", "tc_compress_m257"])
 def test_compress_with_workspace_matches(name):
     """bsa_compress_select_ws (tf32 split once per slab into the workspace) gives bit-identical block
