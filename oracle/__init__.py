@@ -6,6 +6,7 @@ with the CUDA library and imports nothing from it.
 
 Every function works on ONE (batch, head) slab: q, k, v are [N, d], gates
 [N, 3]; inputs are converted to float64 (bf16 values widen exactly).
+backward_slab gives the training gradients of the same forward.
 """
 from __future__ import annotations
 
@@ -41,7 +42,10 @@ def load(path: str | None = None):
                                         _dp, _dp, _dp, _dp, _nullable_d,
                                         _dp, _nullable_d, _nullable_d, _nullable_d,
                                         _nullable_d, _nullable_d, _nullable_d]
-    for f in ("oracle_pool", "oracle_compressed_rows", "oracle_fine_rows", "oracle_forward_slab"):
+    lib.oracle_backward_slab.argtypes = [_i64, _i64, _i64, _i64, _i64, ctypes.c_double,
+                                         _dp, _dp, _dp, _dp, _ip, _dp, _dp, _dp, _dp, _dp]
+    for f in ("oracle_pool", "oracle_compressed_rows", "oracle_fine_rows", "oracle_forward_slab",
+              "oracle_backward_slab"):
         getattr(lib, f).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -149,4 +153,23 @@ def forward_slab(q, k, v, gates, block: int, n: int, w: int, scale: float | None
     return {"out": out, "qbar": qb, "kbar": kb, "vbar": vb, "o_cg": ocg, "idx": idx, "gap": gap}
 
 
-__all__ = ["load", "load_native", "pool", "compressed_rows", "fine_rows", "forward_slab", "default_scale"]
+def backward_slab(q, k, v, gates, idx, dout, block: int, n: int, w: int, scale: float | None = None,
+                  lib=None):
+    """Gradients of one slab's forward with the selection idx [m, n] held fixed.
+
+    dout is dL/dout [N, d]. Returns dict(dq, dk, dv [N, d], dgates [N, 3]).
+    """
+    lib = lib or load()
+    q, k, v, gates, dout = _f64(q), _f64(k), _f64(v), _f64(gates), _f64(dout)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    ntok, d = q.shape
+    scale = default_scale(d) if scale is None else scale
+    dq, dk, dv = (np.empty((ntok, d), np.float64) for _ in range(3))
+    dg = np.empty((ntok, 3), np.float64)
+    rc = lib.oracle_backward_slab(ntok, d, block, n, w, scale, q, k, v, gates, idx, dout, dq, dk, dv, dg)
+    if rc != 0:
+        raise ValueError("oracle_backward_slab: bad arguments")
+    return {"dq": dq, "dk": dk, "dv": dv, "dgates": dg}
+
+
+__all__ = ["load", "load_native", "backward_slab", "pool", "compressed_rows", "fine_rows", "forward_slab", "default_scale"]

@@ -10,6 +10,9 @@
  *   query block keeps the top-n key blocks by compressed score and runs
  *   full-resolution attention over their tokens, (c) local branch: standard
  *   attention over a sliding window, and o = g_CG o_CG + g_FG o_FG + g_L o_L.
+ * The note trains the model through BSA (its loss and training sections), so
+ * the file also holds the backward pass of the same forward: the chain rule
+ * through each step above in reverse, with the block selection held fixed.
  *
  * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or
  * load this file or its library; only the tests, the package's smoke check
@@ -246,5 +249,191 @@ int oracle_forward_slab(int64_t n_tokens, int64_t d, int64_t block, int64_t n, i
         if (gap_out) memcpy(gap_out, gp, (size_t)m * sizeof(double));
     }
     free(qb); free(kb); free(vb); free(ocg); free(ix); free(gp);
+    return rc;
+}
+
+/* ---- backward pass (training) -------------------------------------------- */
+
+/* Gradient of one softmax-attention row over the listed blocks (the reverse
+ * of attend_blocks): with p_u = softmax_u(s q·k_u) and the gradient dO that
+ * reaches this row's output o = sum_u p_u v_u,
+ *   dv_u += p_u dO,   dp_u = dO·v_u,   D = sum_u p_u dp_u,
+ *   ds_u  = p_u (dp_u - D),
+ *   dq_t += s sum_u ds_u k_u,   dk_u += s ds_u q_t.
+ * p and dp are scratch arrays of nb*block doubles. */
+static void attend_blocks_backward(int64_t d, int64_t block, double scale, const double *qt,
+                                   const double *k, const double *v, const int64_t *blocks, int64_t nb,
+                                   const double *dO, double *p, double *dp,
+                                   double *dq_t, double *dk, double *dv)
+{
+    int64_t nk = nb * block;
+    double smax = -INFINITY;
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int64_t t = 0; t < block; ++t) {
+            int64_t u = blocks[b] * block + t;
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += qt[c] * k[u * d + c];
+            p[b * block + t] = scale * dot;
+            if (p[b * block + t] > smax) smax = p[b * block + t];
+        }
+    }
+    double denom = 0.0;
+    for (int64_t e = 0; e < nk; ++e) { p[e] = exp(p[e] - smax); denom += p[e]; }
+    for (int64_t e = 0; e < nk; ++e) p[e] /= denom;
+    double D = 0.0;
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int64_t t = 0; t < block; ++t) {
+            int64_t u = blocks[b] * block + t, e = b * block + t;
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += dO[c] * v[u * d + c];
+            dp[e] = dot;
+            D += p[e] * dot;
+        }
+    }
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int64_t t = 0; t < block; ++t) {
+            int64_t u = blocks[b] * block + t, e = b * block + t;
+            double ds = p[e] * (dp[e] - D);
+            for (int64_t c = 0; c < d; ++c) {
+                dq_t[c] += scale * ds * k[u * d + c];
+                dk[u * d + c] += scale * ds * qt[c];
+                dv[u * d + c] += p[e] * dO[c];
+            }
+        }
+    }
+}
+
+/*
+ * Backward of one slab: given dout = dL/dout [N][d], the gradients dL/dq,
+ * dL/dk, dL/dv [N][d] and dL/dgates [N][3] of the forward pass, with the block
+ * selection idx [m][n] held fixed (the top-n choice is a discrete decision and
+ * carries no gradient). The chain rule through the forward steps in reverse:
+ *   (7) combine: dgates_t = (dout_t·o_CG_i, dout_t·o_FG_t, dout_t·o_L_t); the
+ *       selection and local branches receive g_FG,t dout_t and g_L,t dout_t;
+ *   (5, 6) the selection and local attention rows (attend_blocks_backward);
+ *   (3) compressed branch: dO_CG_i = sum over the tokens t of block i of
+ *       g_CG,t dout_t; with ā_ij = softmax_j(z_ij), dā_ij = dO_CG_i·v̄_j,
+ *       D_i = sum_j ā_ij dā_ij and dz_ij = ā_ij (dā_ij - D_i):
+ *       dq̄_i = s sum_j dz_ij k̄_j,  dk̄_j += s dz_ij q̄_i,  dv̄_j += ā_ij dO_CG_i;
+ *   (2) pooling φ (mean): every token of block j receives 1/B of dq̄_j, dk̄_j, dv̄_j.
+ * A query block whose dout rows are all zero contributes exact zeros to every
+ * sum, so it is skipped. Runs sequentially: the accumulations into dk and dv
+ * from different query blocks happen in query-block order.
+ */
+int oracle_backward_slab(int64_t n_tokens, int64_t d, int64_t block, int64_t n, int64_t w,
+                         double scale, const double *q, const double *k, const double *v,
+                         const double *gates, const int32_t *idx, const double *dout,
+                         double *dq, double *dk, double *dv, double *dgates)
+{
+    if (n_tokens <= 0 || d <= 0 || block <= 0 || n_tokens % block != 0) return -1;
+    int64_t m = n_tokens / block;
+    if (n < 1 || n > m || w < 0) return -1;
+    for (int64_t i = 0; i < m * n; ++i)
+        if (idx[i] < 0 || idx[i] >= m) return -1;
+    int64_t nl_max = 2 * w + 1 < m ? 2 * w + 1 : m;
+    int64_t nmax = (n > nl_max) ? n : nl_max;
+    double *qb = (double *)calloc((size_t)(m * d), sizeof(double));
+    double *kb = (double *)calloc((size_t)(m * d), sizeof(double));
+    double *vb = (double *)calloc((size_t)(m * d), sizeof(double));
+    double *dqb = (double *)calloc((size_t)(m * d), sizeof(double));
+    double *dkb = (double *)calloc((size_t)(m * d), sizeof(double));
+    double *dvb = (double *)calloc((size_t)(m * d), sizeof(double));
+    double *a = (double *)malloc((size_t)m * sizeof(double));
+    double *da = (double *)malloc((size_t)m * sizeof(double));
+    double *ocg = (double *)malloc((size_t)d * sizeof(double));
+    double *docg = (double *)malloc((size_t)d * sizeof(double));
+    double *ofg = (double *)malloc((size_t)d * sizeof(double));
+    double *ol = (double *)malloc((size_t)d * sizeof(double));
+    double *dO = (double *)malloc((size_t)d * sizeof(double));
+    double *p = (double *)malloc((size_t)(nmax * block) * sizeof(double));
+    double *dp = (double *)malloc((size_t)(nmax * block) * sizeof(double));
+    int64_t *sel = (int64_t *)malloc((size_t)n * sizeof(int64_t));
+    int64_t *loc = (int64_t *)malloc((size_t)(2 * w + 1 < m ? 2 * w + 1 : m) * sizeof(int64_t));
+    int rc = -1;
+    if (!qb || !kb || !vb || !dqb || !dkb || !dvb || !a || !da || !ocg || !docg || !ofg || !ol ||
+        !dO || !p || !dp || !sel || !loc)
+        goto done;
+    if (oracle_pool(n_tokens, d, block, q, qb) != 0 || oracle_pool(n_tokens, d, block, k, kb) != 0 ||
+        oracle_pool(n_tokens, d, block, v, vb) != 0)
+        goto done;
+    memset(dq, 0, (size_t)(n_tokens * d) * sizeof(double));
+    memset(dk, 0, (size_t)(n_tokens * d) * sizeof(double));
+    memset(dv, 0, (size_t)(n_tokens * d) * sizeof(double));
+    memset(dgates, 0, (size_t)(n_tokens * 3) * sizeof(double));
+    for (int64_t i = 0; i < m; ++i) {
+        int any = 0;
+        for (int64_t e = i * block * d; e < (i + 1) * block * d; ++e)
+            if (dout[e] != 0.0) { any = 1; break; }
+        if (!any) continue;
+        /* (3) compressed branch, row i: forward probabilities, then its gradients */
+        double zmax = -INFINITY;
+        for (int64_t j = 0; j < m; ++j) {
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += qb[i * d + c] * kb[j * d + c];
+            a[j] = scale * dot;
+            if (a[j] > zmax) zmax = a[j];
+        }
+        double denom = 0.0;
+        for (int64_t j = 0; j < m; ++j) { a[j] = exp(a[j] - zmax); denom += a[j]; }
+        for (int64_t j = 0; j < m; ++j) a[j] /= denom;
+        for (int64_t c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < m; ++j) acc += a[j] * vb[j * d + c];
+            ocg[c] = acc;
+            double g = 0.0;
+            for (int64_t t = i * block; t < (i + 1) * block; ++t) g += gates[t * 3] * dout[t * d + c];
+            docg[c] = g;
+        }
+        double D = 0.0;
+        for (int64_t j = 0; j < m; ++j) {
+            double dot = 0.0;
+            for (int64_t c = 0; c < d; ++c) dot += docg[c] * vb[j * d + c];
+            da[j] = dot;
+            D += a[j] * dot;
+        }
+        for (int64_t j = 0; j < m; ++j) {
+            double dz = a[j] * (da[j] - D);
+            for (int64_t c = 0; c < d; ++c) {
+                dqb[i * d + c] += scale * dz * kb[j * d + c];
+                dkb[j * d + c] += scale * dz * qb[i * d + c];
+                dvb[j * d + c] += a[j] * docg[c];
+            }
+        }
+        /* (5)-(7) the tokens of block i: combine, selection and local branches
+         * (local window: blocks max(0, i-w) .. min(m-1, i+w)) */
+        int64_t lo = i - w, hi = i + w;
+        if (lo < 0) lo = 0;
+        if (hi > m - 1) hi = m - 1;
+        int64_t nl = hi - lo + 1;
+        for (int64_t t = 0; t < n; ++t) sel[t] = (int64_t)idx[i * n + t];
+        for (int64_t b = 0; b < nl; ++b) loc[b] = lo + b;
+        for (int64_t t = i * block; t < (i + 1) * block; ++t) {
+            const double *qt = q + t * d, *g = gates + t * 3, *dy = dout + t * d;
+            attend_blocks(d, block, scale, qt, k, v, sel, n, p, ofg);
+            attend_blocks(d, block, scale, qt, k, v, loc, nl, p, ol);
+            double s0 = 0.0, s1 = 0.0, s2 = 0.0;
+            for (int64_t c = 0; c < d; ++c) { s0 += dy[c] * ocg[c]; s1 += dy[c] * ofg[c]; s2 += dy[c] * ol[c]; }
+            dgates[t * 3] = s0;
+            dgates[t * 3 + 1] = s1;
+            dgates[t * 3 + 2] = s2;
+            for (int64_t c = 0; c < d; ++c) dO[c] = g[1] * dy[c];
+            attend_blocks_backward(d, block, scale, qt, k, v, sel, n, dO, p, dp, dq + t * d, dk, dv);
+            for (int64_t c = 0; c < d; ++c) dO[c] = g[2] * dy[c];
+            attend_blocks_backward(d, block, scale, qt, k, v, loc, nl, dO, p, dp, dq + t * d, dk, dv);
+        }
+    }
+    /* (2) pooling: the mean hands 1/B of each pooled gradient to every token of its block */
+    for (int64_t t = 0; t < n_tokens; ++t) {
+        int64_t j = t / block;
+        for (int64_t c = 0; c < d; ++c) {
+            dq[t * d + c] += dqb[j * d + c] / (double)block;
+            dk[t * d + c] += dkb[j * d + c] / (double)block;
+            dv[t * d + c] += dvb[j * d + c] / (double)block;
+        }
+    }
+    rc = 0;
+done:
+    free(qb); free(kb); free(vb); free(dqb); free(dkb); free(dvb); free(a); free(da);
+    free(ocg); free(docg); free(ofg); free(ol); free(dO); free(p); free(dp); free(sel); free(loc);
     return rc;
 }

@@ -293,6 +293,101 @@ def check_forward_against_masked_dense(lib):
         close(r["out"], want, 1e-12, f"forward vs masked dense (N={n_tok}, B={block}, n={n}, w={w})")
 
 
+# ------------------------------------------------------------------ backward
+
+def _loss_and_forced_forward(lib, q, k, v, g, dout, block, n, w, s, idx):
+    o = oracle.forward_slab(q, k, v, g, block, n, w, scale=s, forced_idx=idx, lib=lib)["out"]
+    return float(np.sum(dout * o))
+
+
+def check_backward_finite_differences(lib):
+    """Central differences of L = sum(dout * out) through the forward oracle (selection held
+    fixed by forcing its indices) against the backward oracle, for every input element."""
+    rng = np.random.default_rng(20)
+    for n_tok, d, block, n, w in ((24, 4, 4, 2, 1), (32, 3, 8, 4, 0)):
+        q, k, v, g = rand_slab(rng, n_tok, d, block)
+        dout = rng.standard_normal((n_tok, d))
+        s = 1.0 / math.sqrt(d)
+        idx = oracle.forward_slab(q, k, v, g, block, n, w, scale=s, lib=lib)["idx"]
+        got = oracle.backward_slab(q, k, v, g, idx, dout, block, n, w, scale=s, lib=lib)
+        h = 1e-5
+        for name, x in (("dq", q), ("dk", k), ("dv", v), ("dgates", g)):
+            num = np.zeros_like(x)
+            for e in range(x.size):
+                old = x.flat[e]
+                x.flat[e] = old + h
+                lp = _loss_and_forced_forward(lib, q, k, v, g, dout, block, n, w, s, idx)
+                x.flat[e] = old - h
+                lm = _loss_and_forced_forward(lib, q, k, v, g, dout, block, n, w, s, idx)
+                x.flat[e] = old
+                num.flat[e] = (lp - lm) / (2 * h)
+            close(got[name], num, 1e-7, f"{name} vs central differences (N={n_tok}, B={block})")
+
+
+def torch_masked_dense_grads(q, k, v, g, dout, block, idx, w, scale):
+    """Gradients of the masked-dense restatement by torch autograd (float64, CPU): pooling by a
+    mean, the compressed branch and both fine branches as library SDPA calls with block masks."""
+    n_tok, d = q.shape
+    m = n_tok // block
+    T = lambda a: torch.tensor(np.asarray(a, np.float64), requires_grad=True)
+    tq, tk, tv, tg = T(q), T(k), T(v), T(g)
+    sdpa = torch.nn.functional.scaled_dot_product_attention
+    qb, kb, vb = (x.reshape(m, block, d).mean(dim=1) for x in (tq, tk, tv))
+    o_cg = sdpa(qb[None, None], kb[None, None], vb[None, None], scale=scale)[0, 0]
+    blk = np.arange(n_tok) // block
+    selb = np.zeros((m, m), bool)
+    np.put_along_axis(selb, np.asarray(idx, np.int64), True, axis=1)
+    sel_mask = torch.from_numpy(selb[blk][:, blk])
+    loc_mask = torch.from_numpy(np.abs(blk[:, None] - blk[None, :]) <= w)
+    o_fg = sdpa(tq[None, None], tk[None, None], tv[None, None], attn_mask=sel_mask[None, None], scale=scale)[0, 0]
+    o_l = sdpa(tq[None, None], tk[None, None], tv[None, None], attn_mask=loc_mask[None, None], scale=scale)[0, 0]
+    out = tg[:, :1] * o_cg[torch.from_numpy(blk)] + tg[:, 1:2] * o_fg + tg[:, 2:3] * o_l
+    grads = torch.autograd.grad(out, (tq, tk, tv, tg), grad_outputs=torch.from_numpy(np.asarray(dout, np.float64)))
+    return {name: x.numpy() for name, x in zip(("dq", "dk", "dv", "dgates"), grads)}
+
+
+def check_backward_against_autograd(lib):
+    """The backward oracle against torch autograd of the masked-dense restatement, including a
+    dout that is zero outside a few query blocks (the oracle skips those blocks)."""
+    rng = np.random.default_rng(21)
+    for n_tok, d, block, n, w, sparse in ((256, 16, 16, 5, 1, False), (192, 8, 4, 48, 0, False),
+                                          (384, 8, 16, 3, 2, True)):
+        q, k, v, g = rand_slab(rng, n_tok, d, block)
+        s = 1.0 / math.sqrt(d)
+        dout = rng.standard_normal((n_tok, d))
+        if sparse:
+            keep = np.zeros(n_tok // block, bool)
+            keep[[1, 7, n_tok // block - 1]] = True
+            dout *= np.repeat(keep, block)[:, None]
+        idx = oracle.forward_slab(q, k, v, g, block, n, w, scale=s, lib=lib)["idx"]
+        got = oracle.backward_slab(q, k, v, g, idx, dout, block, n, w, scale=s, lib=lib)
+        want = torch_masked_dense_grads(q, k, v, g, dout, block, idx, w, s)
+        for name in ("dq", "dk", "dv", "dgates"):
+            close(got[name], want[name], 1e-11, f"{name} vs autograd (N={n_tok}, n={n}, w={w}, sparse={sparse})")
+
+
+def check_backward_linear_in_dout_and_gates(lib):
+    """Gradients are linear in dout; dgates equals dout against each branch's forward output."""
+    rng = np.random.default_rng(22)
+    n_tok, d, block, n, w = 128, 8, 16, 3, 1
+    q, k, v, g = rand_slab(rng, n_tok, d, block)
+    s = 1.0 / math.sqrt(d)
+    fwd = oracle.forward_slab(q, k, v, g, block, n, w, scale=s, lib=lib)
+    a, b = rng.standard_normal((n_tok, d)), rng.standard_normal((n_tok, d))
+    ga = oracle.backward_slab(q, k, v, g, fwd["idx"], a, block, n, w, scale=s, lib=lib)
+    gb = oracle.backward_slab(q, k, v, g, fwd["idx"], b, block, n, w, scale=s, lib=lib)
+    gab = oracle.backward_slab(q, k, v, g, fwd["idx"], 2 * a - 3 * b, block, n, w, scale=s, lib=lib)
+    for name in ("dq", "dk", "dv", "dgates"):
+        close(gab[name], 2 * ga[name] - 3 * gb[name], 1e-12, f"{name} linear in dout")
+    parts = oracle.fine_rows(q, k, v, g, fwd["o_cg"], fwd["idx"], block, n, w, scale=s, want_branches=True, lib=lib)
+    cg_tok = np.repeat(fwd["o_cg"], block, axis=0)
+    want = np.stack([np.sum(a * cg_tok, 1), np.sum(a * parts["o_fg"], 1), np.sum(a * parts["o_l"], 1)], 1)
+    close(ga["dgates"], want, 1e-13, "dgates = dout against the branch outputs")
+    zero = oracle.backward_slab(q, k, v, g, fwd["idx"], np.zeros((n_tok, d)), block, n, w, scale=s, lib=lib)
+    for name in ("dq", "dk", "dv", "dgates"):
+        assert not np.any(zero[name]), f"{name} must vanish for dout = 0"
+
+
 ALL_CHECKS = [
     check_pool_partition_is_nested_parent,
     check_pool_constant_and_linear,
@@ -305,4 +400,7 @@ ALL_CHECKS = [
     check_gates_and_constant_values,
     check_forced_index_permutation,
     check_forward_against_masked_dense,
+    check_backward_finite_differences,
+    check_backward_against_autograd,
+    check_backward_linear_in_dout_and_gates,
 ]

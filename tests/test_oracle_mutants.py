@@ -32,6 +32,22 @@ MUTANTS = {
     "gates_fg_l_swapped": ("g[1] * ofg[c] + g[2] * ol[c]", "g[2] * ofg[c] + g[1] * ol[c]"),
     "cg_term_dropped": ("g[0] * o_cg[i * d + c] + g[1]", "0.0 * o_cg[i * d + c] + g[1]"),
     "cg_wrong_block": ("g[0] * o_cg[i * d + c]", "g[0] * o_cg[(m - 1 - i) * d + c]"),
+    # backward
+    "bwd_fine_D_dropped": ("double ds = p[e] * (dp[e] - D);", "double ds = p[e] * dp[e];"),
+    "bwd_dk_no_scale": ("dk[u * d + c] += scale * ds * qt[c];", "dk[u * d + c] += ds * qt[c];"),
+    "bwd_dv_uses_dp": ("dv[u * d + c] += p[e] * dO[c];", "dv[u * d + c] += dp[e] * dO[c];"),
+    "bwd_dq_uses_v": ("dq_t[c] += scale * ds * k[u * d + c];", "dq_t[c] += scale * ds * v[u * d + c];"),
+    "bwd_compressed_D_dropped": ("double dz = a[j] * (da[j] - D);", "double dz = a[j] * da[j];"),
+    "bwd_dkbar_uses_kbar": ("dkb[j * d + c] += scale * dz * qb[i * d + c];", "dkb[j * d + c] += scale * dz * kb[i * d + c];"),
+    "bwd_docg_wrong_gate": ("g += gates[t * 3] * dout[t * d + c];", "g += gates[t * 3 + 1] * dout[t * d + c];"),
+    "bwd_local_gets_fg_gate": ("dO[c] = g[2] * dy[c];", "dO[c] = g[1] * dy[c];"),
+    "bwd_pool_grad_not_divided": ("dk[t * d + c] += dkb[j * d + c] / (double)block;", "dk[t * d + c] += dkb[j * d + c];"),
+    "bwd_dgates_swapped": ("dgates[t * 3 + 1] = s1;\n            dgates[t * 3 + 2] = s2;",
+                           "dgates[t * 3 + 1] = s2;\n            dgates[t * 3 + 2] = s1;"),
+    "bwd_window_right_edge_dropped": ("int64_t lo = i - w, hi = i + w;", "int64_t lo = i - w, hi = i;"),
+    "bwd_window_wraps_left": ("if (lo < 0) lo = 0;", "if (lo < 0) lo = i;"),
+    "bwd_selection_uses_row0": ("sel[t] = (int64_t)idx[i * n + t];", "sel[t] = (int64_t)idx[t];"),
+    "bwd_softmax_not_normalised": ("for (int64_t e = 0; e < nk; ++e) p[e] /= denom;", "(void)denom;"),
 }
 
 
