@@ -44,8 +44,12 @@ def load(path: str | None = None):
                                         _nullable_d, _nullable_d, _nullable_d]
     lib.oracle_backward_slab.argtypes = [_i64, _i64, _i64, _i64, _i64, ctypes.c_double,
                                          _dp, _dp, _dp, _dp, _ip, _dp, _dp, _dp, _dp, _dp]
+    lib.oracle_healpix_center.argtypes = [_i64, _i64, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]
+    lib.oracle_healpix_center.restype = None
+    lib.oracle_latlon_plan.argtypes = [_i64, _i64, _i64, _ip, _dp]
+    lib.oracle_interp.argtypes = [_i64, _i64, _i64, _i64, ctypes.c_double, _ip, _dp, _dp, _dp, _dp, _dp]
     for f in ("oracle_pool", "oracle_compressed_rows", "oracle_fine_rows", "oracle_forward_slab",
-              "oracle_backward_slab"):
+              "oracle_backward_slab", "oracle_latlon_plan", "oracle_interp"):
         getattr(lib, f).restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -172,4 +176,42 @@ def backward_slab(q, k, v, gates, idx, dout, block: int, n: int, w: int, scale: 
     return {"dq": dq, "dk": dk, "dv": dv, "dgates": dg}
 
 
-__all__ = ["load", "load_native", "backward_slab", "pool", "compressed_rows", "fine_rows", "forward_slab", "default_scale"]
+def healpix_centers(nside: int, lib=None) -> np.ndarray:
+    """(z, phi) of every NESTED pixel centre at nside -> [12 nside^2, 2]."""
+    lib = lib or load()
+    n = 12 * nside * nside
+    out = np.empty((n, 2), np.float64)
+    z, ph = ctypes.c_double(), ctypes.c_double()
+    for p in range(n):
+        lib.oracle_healpix_center(nside, p, ctypes.byref(z), ctypes.byref(ph))
+        out[p] = (z.value, ph.value)
+    return out
+
+
+def latlon_plan(nside: int, nlat: int, nlon: int, lib=None):
+    """4 x 4 lat-lon neighbourhood (source indices [npix, 16]) and relative positions [npix, 16, 3]."""
+    lib = lib or load()
+    n = 12 * nside * nside
+    nbr = np.empty((n, 16), np.int32)
+    rel = np.empty((n, 16, 3), np.float64)
+    if lib.oracle_latlon_plan(nside, nlat, nlon, nbr, rel) != 0:
+        raise ValueError("oracle_latlon_plan: bad arguments")
+    return nbr, rel
+
+
+def interp(nbr, rel, wq, ksrc, vsrc, scale: float | None = None, lib=None) -> np.ndarray:
+    """Cross-attention interpolation: out [n_tgt, d] from neighbours nbr [n_tgt, K], positions
+    rel [n_tgt, K, 3], query map wq [d, 3] and source keys/values [n_src, d]."""
+    lib = lib or load()
+    nbr = np.ascontiguousarray(nbr, np.int32)
+    rel, wq, ksrc, vsrc = _f64(rel), _f64(wq), _f64(ksrc), _f64(vsrc)
+    n_tgt, K = nbr.shape
+    n_src, d = ksrc.shape
+    scale = default_scale(d) if scale is None else scale
+    out = np.empty((n_tgt, d), np.float64)
+    if lib.oracle_interp(n_tgt, K, d, n_src, scale, nbr, rel, wq, ksrc, vsrc, out) != 0:
+        raise ValueError("oracle_interp: bad arguments")
+    return out
+
+
+__all__ = ["load", "load_native", "backward_slab", "healpix_centers", "latlon_plan", "interp", "pool", "compressed_rows", "fine_rows", "forward_slab", "default_scale"]

@@ -388,6 +388,96 @@ def check_backward_linear_in_dout_and_gates(lib):
         assert not np.any(zero[name]), f"{name} must vanish for dout = 0"
 
 
+# ------------------------------------------- lat-lon -> HEALPix interpolation
+
+def ring_scheme_centres(nside):
+    """Pixel centres listed ring by ring (the published HEALPix ring formulas), no faces or bits."""
+    pts = []
+    for i in range(1, 4 * nside):
+        if i < nside:
+            nr, z, s = i, 1 - i * i / (3 * nside * nside), 1
+        elif i > 3 * nside:
+            nr = 4 * nside - i
+            z, s = -1 + nr * nr / (3 * nside * nside), 1
+        else:
+            nr, z, s = nside, 4 / 3 - 2 * i / (3 * nside), (i - nside + 1) % 2
+        for j in range(1, 4 * nr + 1):
+            pts.append((z, ((j - s / 2) * math.pi / (2 * nr)) % (2 * math.pi)))
+    return np.array(pts)
+
+
+def unit(zphi):
+    z, ph = zphi[:, 0], zphi[:, 1]
+    st = np.sqrt(1 - z * z)
+    return np.stack([st * np.cos(ph), st * np.sin(ph), z], 1)
+
+
+def check_healpix_centres(lib):
+    """NESTED centres: the 12 base pixels, the same point set as the ring-by-ring listing, equal
+    area (mean z^2 of a uniform sphere sample tends to 1/3), and the child rule 4p..4p+3 (the
+    four children of p surround p's centre)."""
+    c1 = oracle.healpix_centers(1, lib=lib)
+    want_z = [2 / 3] * 4 + [0] * 4 + [-2 / 3] * 4
+    want_phi = [math.pi / 4 * (2 * f + 1) for f in range(4)] + [math.pi / 2 * f for f in range(4)] + \
+               [math.pi / 4 * (2 * f + 1) for f in range(4)]
+    close(c1[:, 0], want_z, 1e-15, "base pixel z")
+    close(c1[:, 1], want_phi, 1e-15, "base pixel phi")
+    for nside in (2, 4, 8, 16):
+        c = oracle.healpix_centers(nside, lib=lib)
+        assert len(c) == 12 * nside * nside
+        key = lambda a: sorted((round(z, 12), round(p, 12)) for z, p in a)
+        assert key(c) == key(ring_scheme_centres(nside)), f"centres differ from the ring listing (nside {nside})"
+        assert abs(float(np.mean(c[:, 0] ** 2)) - 1 / 3) < 0.2 / nside ** 2 + 1e-3
+        fine = unit(oracle.healpix_centers(2 * nside, lib=lib)).reshape(-1, 4, 3)
+        parent = unit(c)
+        mean_child = fine.mean(axis=1)
+        mean_child /= np.linalg.norm(mean_child, axis=1, keepdims=True)
+        ang = np.degrees(np.arccos(np.clip(np.sum(mean_child * parent, 1), -1, 1)))
+        assert ang.max() < 0.5 * 58.63 / nside, f"children 4p..4p+3 not around p (nside {nside}: {ang.max():.2f} deg)"
+
+
+def check_latlon_plan(lib):
+    """Every neighbourhood holds 16 distinct grid points including the target's nearest grid point
+    (brute force over the whole grid), and the relative positions are the unit-vector differences
+    over the grid step."""
+    for nside, nlat, nlon in ((4, 25, 48), (8, 19, 36), (2, 7, 12)):
+        nbr, rel = oracle.latlon_plan(nside, nlat, nlon, lib=lib)
+        tgt = unit(oracle.healpix_centers(nside, lib=lib))
+        dlat = 180 / (nlat - 1)
+        lat = np.radians(90 - dlat * np.arange(nlat))
+        lon = np.radians(360 / nlon * np.arange(nlon))
+        src = np.stack([np.cos(lat)[:, None] * np.cos(lon)[None, :], np.cos(lat)[:, None] * np.sin(lon)[None, :],
+                        np.broadcast_to(np.sin(lat)[:, None], (nlat, nlon))], -1).reshape(-1, 3)
+        nearest = np.argmax(tgt @ src.T, axis=1)
+        for i in range(len(tgt)):
+            assert len(set(nbr[i].tolist())) == 16, f"pixel {i}: repeated neighbours"
+            assert nearest[i] in set(nbr[i].tolist()) or np.isclose(
+                (tgt[i] @ src[nearest[i]]), max(tgt[i] @ src[j] for j in nbr[i]), atol=1e-12), \
+                f"pixel {i}: nearest grid point not in its neighbourhood"
+        close(rel, (src[nbr] - tgt[:, None, :]) / np.radians(dlat), 1e-12, "relative positions")
+
+
+def check_interp(lib):
+    """The interpolation against (a) the logits formed the other way round, q_ij . k_j =
+    p_ij . (W_q^T k_j), with a library softmax; (b) W_q = 0: the plain mean of the neighbours'
+    values; (c) one neighbour set repeated: the value itself."""
+    rng = np.random.default_rng(23)
+    n_src, d, K, n_tgt = 40, 16, 16, 30
+    nbr = np.stack([rng.choice(n_src, K, replace=False) for _ in range(n_tgt)]).astype(np.int32)
+    rel = rng.standard_normal((n_tgt, K, 3))
+    wq = rng.standard_normal((d, 3))
+    ks, vs = rng.standard_normal((n_src, d)), rng.standard_normal((n_src, d))
+    s = 1 / math.sqrt(d)
+    got = oracle.interp(nbr, rel, wq, ks, vs, lib=lib)
+    kappa = ks @ wq                                   # [n_src, 3]: keys seen from position space
+    logits = s * np.einsum("ike,ike->ik", rel, kappa[nbr])
+    p = torch.softmax(torch.from_numpy(logits), dim=1).numpy()
+    close(got, np.einsum("ik,ikc->ic", p, vs[nbr]), 1e-13, "interp vs position-space logits")
+    close(oracle.interp(nbr, rel, np.zeros((d, 3)), ks, vs, lib=lib), vs[nbr].mean(axis=1), 1e-14, "W_q = 0 mean")
+    one = np.repeat(nbr[:, :1], K, axis=1)
+    close(oracle.interp(one, rel, wq, ks, vs, lib=lib), vs[nbr[:, 0]], 1e-14, "single source")
+
+
 ALL_CHECKS = [
     check_pool_partition_is_nested_parent,
     check_pool_constant_and_linear,
@@ -403,4 +493,7 @@ ALL_CHECKS = [
     check_backward_finite_differences,
     check_backward_against_autograd,
     check_backward_linear_in_dout_and_gates,
+    check_healpix_centres,
+    check_latlon_plan,
+    check_interp,
 ]

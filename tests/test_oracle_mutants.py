@@ -38,15 +38,30 @@ MUTANTS = {
     "bwd_dv_uses_dp": ("dv[u * d + c] += p[e] * dO[c];", "dv[u * d + c] += dp[e] * dO[c];"),
     "bwd_dq_uses_v": ("dq_t[c] += scale * ds * k[u * d + c];", "dq_t[c] += scale * ds * v[u * d + c];"),
     "bwd_compressed_D_dropped": ("double dz = a[j] * (da[j] - D);", "double dz = a[j] * da[j];"),
-    "bwd_dkbar_uses_kbar": ("dkb[j * d + c] += scale * dz * qb[i * d + c];", "dkb[j * d + c] += scale * dz * kb[i * d + c];"),
+    "bwd_dkbar_uses_kbar": ("dkb_p[j * d + c] += scale * dz * qb[i * d + c];",
+                            "dkb_p[j * d + c] += scale * dz * kb[i * d + c];"),
     "bwd_docg_wrong_gate": ("g += gates[t * 3] * dout[t * d + c];", "g += gates[t * 3 + 1] * dout[t * d + c];"),
     "bwd_local_gets_fg_gate": ("dO[c] = g[2] * dy[c];", "dO[c] = g[1] * dy[c];"),
     "bwd_pool_grad_not_divided": ("dk[t * d + c] += dkb[j * d + c] / (double)block;", "dk[t * d + c] += dkb[j * d + c];"),
-    "bwd_dgates_swapped": ("dgates[t * 3 + 1] = s1;\n            dgates[t * 3 + 2] = s2;",
-                           "dgates[t * 3 + 1] = s2;\n            dgates[t * 3 + 2] = s1;"),
+    "bwd_dgates_fg_gets_l": ("dgates[t * 3 + 1] = s1;", "dgates[t * 3 + 1] = s2;"),
     "bwd_window_right_edge_dropped": ("int64_t lo = i - w, hi = i + w;", "int64_t lo = i - w, hi = i;"),
     "bwd_window_wraps_left": ("if (lo < 0) lo = 0;", "if (lo < 0) lo = i;"),
     "bwd_selection_uses_row0": ("sel[t] = (int64_t)idx[i * n + t];", "sel[t] = (int64_t)idx[t];"),
+    # lat-lon -> HEALPix interpolation
+    "hp_ring_off_by_one": ("int64_t ring = face_row[f] * nside - x - y - 1;", "int64_t ring = face_row[f] * nside - x - y;"),
+    "hp_equatorial_z": ("*z = 4.0 / 3.0 - 2.0 * (double)ring / (3.0 * (double)nside);",
+                        "*z = 1.0 - 2.0 * (double)ring / (3.0 * (double)nside);"),
+    "hp_face_columns_shifted": ("static const int face_col[12] = {1, 3, 5, 7, 0, 2, 4, 6, 1, 3, 5, 7};",
+                                "static const int face_col[12] = {1, 3, 5, 7, 1, 3, 5, 7, 1, 3, 5, 7};"),
+    "hp_bits_not_interleaved": ("y |= ((ipf >> (2 * b + 1)) & 1) << b;", "y |= ((ipf >> (2 * b + 1)) & 1) << (b + 1);"),
+    "plan_window_off_by_one": ("int64_t r = r0 + a, c = ((c0 - 1 + b) % nlon + nlon) % nlon;",
+                               "int64_t r = r0 + a, c = ((c0 + 1 + b) % nlon + nlon) % nlon;"),
+    "plan_rel_unscaled": ("rel[e * 3 + t] = (xj[t] - xi[t]) / h;", "rel[e * 3 + t] = (xj[t] - xi[t]);"),
+    "interp_not_normalised": ("out[i * d + c] = acc / denom;", "out[i * d + c] = acc;"),
+    "interp_values_are_keys": ("acc += s[j] * vsrc[(int64_t)nbr[i * K + j] * d + c];",
+                               "acc += s[j] * ksrc[(int64_t)nbr[i * K + j] * d + c];"),
+    "interp_query_column": ("double qc = wq[c * 3] * p[0] + wq[c * 3 + 1] * p[1] + wq[c * 3 + 2] * p[2];",
+                            "double qc = wq[c * 3] * p[0] + wq[c * 3 + 1] * p[2] + wq[c * 3 + 2] * p[1];"),
     "bwd_softmax_not_normalised": ("for (int64_t e = 0; e < nk; ++e) p[e] /= denom;", "(void)denom;"),
 }
 
