@@ -46,7 +46,7 @@ TF32_PER_BF16 = 1.1 / 2.25     # nominal dense tf32 : bf16 tensor rate (B200)
 
 def compress_on_tensor_cores(cfg) -> bool:
     """The library runs the compressed branch on the tensor cores (three-pass tf32) for these shapes."""
-    return cfg.head_dim == 64 and cfg.top_n == 16
+    return cfg.head_dim == 64 and cfg.top_n in (16, 32)
 
 
 def kernels_per_step(cfg) -> int:
@@ -461,6 +461,126 @@ def run_ours(args, cfg, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_sharded(args, cfg, rank, world, local_rank):
+    """One problem split by (batch, head) slab over the ranks (sharding.ShardedBSA): each rank runs
+    bsa_forward on its contiguous slab range, then one NCCL all-gather reassembles the output on
+    every rank. A step = shard forward + all-gather; "scaling": "strong" (the job's work is fixed)."""
+    import torch
+    import torch.distributed as dist
+    from block_sparse_spherical_b200.replicas import barrier, max_over_ranks
+    from block_sparse_spherical_b200.sharding import ShardedBSA
+    from block_sparse_spherical_b200.synthetic import make_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    qh, kh, vh, gh = make_inputs(cfg)
+    host = lambda a: torch.from_numpy(a).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+    q, k, v, g = (host(a).to(dev) for a in (qh, kh, vh, gh))
+    layer = ShardedBSA(cfg.batch, cfg.heads, cfg.n_tokens, cfg.head_dim, cfg.block_size, cfg.top_n,
+                       cfg.window_blocks, torch.bfloat16 if cfg.dtype == "bf16" else torch.float32, device=dev,
+                       gather="fused" if args.fused_gather else "nccl")
+    for _ in range(args.warmup):
+        layer(q, k, v, g)
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for _ in range(args.steps):
+        layer(q, k, v, g)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    total_ms = max_over_ranks(a.elapsed_time(b), dev)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    ms = total_ms / args.steps
+    line = {"metric": METRIC, "mode": "sharded", "value": cfg.batch * cfg.n_tokens / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": cfg.dtype,
+            "data": "synthetic",
+            "config": dict(workload_config(cfg), parallelism=f"(batch, head) slabs split over {world} rank(s) + "
+                                                             + ("output rows stored to every rank by the kernel"
+                                                                if args.fused_gather else "NCCL all-gather of the output")),
+            "tflops": (cfg.fine_flops() + cfg.compressed_flops()) / (ms / 1e3) / 1e12,
+            "gpu_launches": 4 * args.steps, "gpu": torch.cuda.get_device_name(dev)}
+    print(json.dumps(line), flush=True)
+
+
+def run_backward(args, cfg, rank, world, local_rank):
+    """Training pass: one step = bsa_backward (every backward kernel) on the saved tensors of one
+    bsa_forward_train of the workload, with a seeded dout; the forward itself is not timed."""
+    import torch
+    import torch.distributed as dist
+    from block_sparse_spherical_b200 import abi, api
+    from block_sparse_spherical_b200.replicas import barrier, job_tokens_per_step, max_over_ranks, replica_config
+    from block_sparse_spherical_b200.synthetic import f32_to_bf16_bits, make_inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    rcfg = replica_config(cfg, rank)
+    qh, kh, vh, gh = make_inputs(rcfg)
+    host = lambda a: torch.from_numpy(a).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+    q, k, v, g = (host(a).to(dev) for a in (qh, kh, vh, gh))
+    rng = np.random.default_rng(rcfg.seed + 77)
+    dout = host(f32_to_bf16_bits(rng.standard_normal(qh.shape, dtype=np.float32))).to(dev)
+    layer = api.BSATrain.from_config(cfg, device=dev)
+    layer(q, k, v, g)
+    grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(g))
+    for _ in range(args.warmup):
+        layer.backward(dout, grads)
+    torch.cuda.synchronize(dev)
+    if layer.check_status() != 0 or layer.check_backward_status() != 0:
+        raise RuntimeError("kernel status word reports an error")
+    stream = torch.cuda.current_stream(dev)
+    sampler = ClockSampler(None) if rank == 0 else None
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.5)
+    a.record(stream)
+    for _ in range(args.steps):
+        layer.backward(dout, grads)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    total_ms = max_over_ranks(a.elapsed_time(b), dev)
+    if layer.check_backward_status() != 0:
+        raise RuntimeError("kernel status word reports an error")
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    ms = total_ms / args.steps
+    # algorithmic work: per (query, key) pair the backward recomputes S and forms dP, dV, dK and dQ,
+    # 10*d flops against the forward's 4*d, in both the fine branches and the compressed branch
+    flops = 2.5 * (cfg.fine_flops() + cfg.compressed_flops())
+    tf = world * flops / (ms / 1e3) / 1e12
+    line = {"metric": "BSA bwd tokens/s & TFLOP/s (training gradient of the forward; selection held fixed)",
+            "pass": "backward", "value": job_tokens_per_step(cfg, world) / (ms / 1e3), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+            "data": "synthetic", "config": dict(workload_config(cfg), parallelism=f"{world} independent replica(s)"),
+            "tflops": tf, "algorithmic_flops": flops,
+            "roofline": {"kernel": "whole backward (10 kernels; attend_bwd_tc dominant, see profiles/)",
+                         "bound": "tensor", "achieved": tf / world, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tf / world / peaks["bf16_tflops"], "peak_source": f"{peak_src} bf16_tflops (burst)",
+                         "traffic": None},
+            "gpu_launches": 10 * args.steps, "clocks": clocks, "gpu": torch.cuda.get_device_name(dev)}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -470,6 +590,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
+                    help="backward: time the training gradient (bsa_backward) instead of the forward")
+    ap.add_argument("--shard", action="store_true",
+                    help="split one problem's (batch, head) slabs over the ranks (strong scaling) instead of "
+                         "running an independent replica per rank")
+    ap.add_argument("--fused-gather", action="store_true",
+                    help="with --shard: the kernel's epilogue stores output rows into every rank's buffer "
+                         "(symmetric memory) instead of an NCCL all-gather after the forward")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -479,6 +607,10 @@ def main():
     cfg = CONFIGS[args.workload]
     if args.impl == "reference":
         run_reference(args, cfg, rank)
+    elif args.which == "backward":
+        run_backward(args, cfg, rank, world, local_rank)
+    elif args.shard:
+        run_sharded(args, cfg, rank, world, local_rank)
     else:
         run_ours(args, cfg, rank, world, local_rank)
 

@@ -20,8 +20,10 @@ STATUS_NAMES = {
     4: "BSA_ERR_CUDA", 5: "BSA_ERR_TIMEOUT", 6: "BSA_ERR_WORKSPACE", 7: "BSA_ERR_INDEX",
 }
 EXPORTS = ("bsa_pool", "bsa_compress_select", "bsa_compress_select_ws", "bsa_fine_attention",
-           "bsa_workspace_size", "bsa_forward", "bsa_check_status", "bsa_status_string", "bsa_forward_noalloc")
-TESTING_EXPORTS = ("bsa_testing_fine_attention_withhold",)
+           "bsa_workspace_size", "bsa_forward", "bsa_check_status", "bsa_status_string", "bsa_forward_noalloc",
+           "bsa_forward_train", "bsa_backward_workspace_size", "bsa_backward", "bsa_permute_tokens",
+           "bsa_latlon_healpix_plan", "bsa_latlon_to_healpix", "bsa_forward_mirrored")
+TESTING_EXPORTS = ("bsa_testing_fine_attention_withhold", "bsa_testing_exp2")
 
 
 class BsaConfig(ctypes.Structure):
@@ -58,7 +60,16 @@ def load() -> ctypes.CDLL:
         "bsa_check_status": [P, P],
         "bsa_status_string": [ctypes.c_int],
         "bsa_forward_noalloc": [C, P, P, P, P, P, P, P, P],
+        "bsa_forward_train": [C, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
+        "bsa_backward_workspace_size": [C, ctypes.POINTER(ctypes.c_size_t)],
+        "bsa_backward": [C, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P],
+        "bsa_permute_tokens": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P, P, P, P],
+        "bsa_latlon_healpix_plan": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P, P],
+        "bsa_forward_mirrored": [C, P, P, P, P, P, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, P, P, S, P],
+        "bsa_latlon_to_healpix": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                                  ctypes.c_float, P, P, P, P, P, P, P, P],
         "bsa_testing_fine_attention_withhold": [C, P, P, P, P, P, P, P, P, ctypes.c_int64, P],
+        "bsa_testing_exp2": [P, P, ctypes.c_int64, ctypes.c_int32, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -138,6 +149,53 @@ def bsa_forward_noalloc(cfg: BsaConfig, q, k, v, gates, out, sel_idx_out=None, s
     _check("bsa_forward_noalloc", load().bsa_forward_noalloc(
         ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(out), _ptr(sel_idx_out),
         _ptr(status_word), _stream(stream)))
+
+
+def bsa_forward_train(cfg: BsaConfig, q, k, v, gates, out, sel_idx, o_cg_block, lse_cg, o_fg, o_l, lse_fine,
+                      workspace, workspace_bytes: int, stream=None) -> None:
+    _check("bsa_forward_train", load().bsa_forward_train(
+        ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(out), _ptr(sel_idx), _ptr(o_cg_block),
+        _ptr(lse_cg), _ptr(o_fg), _ptr(o_l), _ptr(lse_fine), _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def bsa_backward_workspace_size(cfg: BsaConfig) -> int:
+    n = ctypes.c_size_t(0)
+    _check("bsa_backward_workspace_size", load().bsa_backward_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def bsa_backward(cfg: BsaConfig, q, k, v, gates, dout, sel_idx, o_cg_block, lse_cg, o_fg, o_l, lse_fine,
+                 dq, dk, dv, dgates, workspace, workspace_bytes: int, stream=None) -> None:
+    _check("bsa_backward", load().bsa_backward(
+        ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(dout), _ptr(sel_idx), _ptr(o_cg_block),
+        _ptr(lse_cg), _ptr(o_fg), _ptr(o_l), _ptr(lse_fine), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgates),
+        _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def bsa_permute_tokens(slabs: int, n_tokens: int, row_bytes: int, perm, src, dst, status_word=None,
+                       stream=None) -> None:
+    _check("bsa_permute_tokens", load().bsa_permute_tokens(slabs, n_tokens, row_bytes, _ptr(perm), _ptr(src),
+                                                           _ptr(dst), _ptr(status_word), _stream(stream)))
+
+
+def bsa_latlon_healpix_plan(nside: int, nlat: int, nlon: int, nbr, rel, stream=None) -> None:
+    _check("bsa_latlon_healpix_plan", load().bsa_latlon_healpix_plan(nside, nlat, nlon, _ptr(nbr), _ptr(rel),
+                                                                     _stream(stream)))
+
+
+def bsa_latlon_to_healpix(batch: int, n_tgt: int, n_src: int, head_dim: int, dtype: int, scale: float, nbr, rel,
+                          wq, k_src, v_src, out, status_word=None, stream=None) -> None:
+    _check("bsa_latlon_to_healpix", load().bsa_latlon_to_healpix(
+        batch, n_tgt, n_src, head_dim, dtype, scale, _ptr(nbr), _ptr(rel), _ptr(wq), _ptr(k_src), _ptr(v_src),
+        _ptr(out), _ptr(status_word), _stream(stream)))
+
+
+def bsa_forward_mirrored(cfg: BsaConfig, q, k, v, gates, out, mirrors, sel_idx_out, workspace,
+                         workspace_bytes: int, stream=None) -> None:
+    arr = (ctypes.c_void_p * max(1, len(mirrors)))(*[_ptr(m) for m in mirrors])
+    _check("bsa_forward_mirrored", load().bsa_forward_mirrored(
+        ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(out), arr, len(mirrors),
+        _ptr(sel_idx_out), _ptr(workspace), workspace_bytes, _stream(stream)))
 
 
 def bsa_check_status(status_word, stream=None) -> int:

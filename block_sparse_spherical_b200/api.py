@@ -76,6 +76,90 @@ class BSA:
         return abi.bsa_check_status(self.workspace)
 
 
+class BSATrain(BSA):
+    """A BSA layer of fixed shape for training: forward() saves what backward() needs.
+
+    forward(q, k, v, gates) -> out; backward(dout) -> (dq, dk, dv, dgates), with the
+    selected blocks held fixed. bf16, block 64, head_dim 64. The saved tensors and
+    both workspaces live on the device between the two calls.
+    """
+
+    def __init__(self, *args, **kw):
+        super().__init__(*args, **kw)
+        b, h, n, d = self.shape
+        dev = self.workspace.device
+        self.o_cg = torch.empty((b, h, self.m, d), dtype=torch.float32, device=dev)
+        self.lse_cg = torch.empty((b, h, self.m), dtype=torch.float32, device=dev)
+        self.o_fg = torch.empty(self.shape, dtype=self.dtype, device=dev)
+        self.o_l = torch.empty(self.shape, dtype=self.dtype, device=dev)
+        self.lse_fine = torch.empty((b, h, n, 2), dtype=torch.float32, device=dev)
+        self.bwd_workspace_bytes = abi.bsa_backward_workspace_size(self.cfg)
+        self.bwd_workspace = torch.zeros(self.bwd_workspace_bytes, dtype=torch.uint8, device=dev)
+        self._saved = None
+
+    def __call__(self, q, k, v, gates, out=None) -> torch.Tensor:
+        return self.forward(q, k, v, gates, out)
+
+    def forward(self, q, k, v, gates, out=None) -> torch.Tensor:
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            _require(t, name, self.dtype, self.shape)
+        _require(gates, "gates", torch.float32, self.shape[:3] + (3,))
+        if out is None:
+            out = torch.empty_like(q)
+        _require(out, "out", self.dtype, self.shape)
+        abi.bsa_forward_train(self.cfg, q, k, v, gates, out, self.sel_idx, self.o_cg, self.lse_cg, self.o_fg,
+                              self.o_l, self.lse_fine, self.workspace, self.workspace_bytes)
+        self._saved = (q, k, v, gates)
+        return out
+
+    def backward(self, dout, grads=None):
+        """Gradients (dq, dk, dv, dgates) of the last forward() for dL/dout = dout."""
+        if self._saved is None:
+            raise RuntimeError("backward() needs a forward() first")
+        q, k, v, gates = self._saved
+        _require(dout, "dout", self.dtype, self.shape)
+        if grads is None:
+            grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(gates))
+        dq, dk, dv, dg = grads
+        abi.bsa_backward(self.cfg, q, k, v, gates, dout, self.sel_idx, self.o_cg, self.lse_cg, self.o_fg, self.o_l,
+                         self.lse_fine, dq, dk, dv, dg, self.bwd_workspace, self.bwd_workspace_bytes)
+        return dq, dk, dv, dg
+
+    def check_backward_status(self) -> int:
+        """Synchronise and return the backward kernels' status code (0 = OK); resets it."""
+        return abi.bsa_check_status(self.bwd_workspace)
+
+
+class LatLonToHealpix:
+    """Cross-attention interpolation from a lat-lon grid to the HEALPix NESTED pixels at nside.
+
+    The plan (16 neighbours and relative positions per pixel) is built once on the
+    device; calling the object with k_src, v_src [B, nlat*nlon, d] (bf16 or fp32) and
+    the query map wq [d, 3] (fp32) returns [B, 12*nside^2, d].
+    """
+
+    def __init__(self, nside: int, nlat: int, nlon: int, device="cuda"):
+        self.nside, self.nlat, self.nlon = nside, nlat, nlon
+        self.npix = 12 * nside * nside
+        self.nbr = torch.empty((self.npix, 16), dtype=torch.int32, device=device)
+        self.rel = torch.empty((self.npix, 16, 3), dtype=torch.float32, device=device)
+        abi.bsa_latlon_healpix_plan(nside, nlat, nlon, self.nbr, self.rel)
+
+    def __call__(self, k_src, v_src, wq, scale: float = 0.0, out=None, status_word=None):
+        b, n_src, d = k_src.shape
+        if n_src != self.nlat * self.nlon:
+            raise ValueError(f"k_src must hold {self.nlat * self.nlon} grid points, got {n_src}")
+        _require(k_src, "k_src")
+        _require(v_src, "v_src", k_src.dtype, k_src.shape)
+        _require(wq, "wq", torch.float32, (d, 3))
+        if out is None:
+            out = torch.empty((b, self.npix, d), dtype=k_src.dtype, device=k_src.device)
+        _require(out, "out", k_src.dtype, (b, self.npix, d))
+        abi.bsa_latlon_to_healpix(b, self.npix, n_src, d, _dtype_code(k_src), scale, self.nbr, self.rel, wq, k_src,
+                                  v_src, out, status_word)
+        return out
+
+
 def forward(q, k, v, gates, block_size: int, top_n: int, window_blocks: int = 1, scale: float = 0.0,
             return_indices: bool = False):
     """One-shot BSA forward (allocates a workspace; use BSA for repeated calls)."""

@@ -62,9 +62,15 @@ constexpr int TILE = BK * HD * 2;           // bytes of one 64x64 bf16 tile
 #ifndef BSA_TC_P_TMEM
 #define BSA_TC_P_TMEM 1
 #endif
+#ifndef BSA_TC_POLY_PAIRS
+#define BSA_TC_POLY_PAIRS 0
+#endif
 constexpr int NSLOT = BSA_TC_SLOTS;        // independent pipelines per CTA
 constexpr int NSTAGE = BSA_TC_STAGES;      // depth of the K and V rings
 constexpr bool P_TMEM = BSA_TC_P_TMEM != 0;   // P·V reads P from tensor memory (else shared memory)
+// of each thread's 16 pairs of softmax numerators per step, how many take the FMA-pipe exp2
+// (exp2_poly2) instead of the exp unit (ex2.approx), to share the load between the two pipes
+constexpr int POLY_PAIRS = BSA_TC_POLY_PAIRS;
 constexpr int NTHREADS = 32 * (2 * NSLOT + 4 * NSLOT);
 // Register split (setmaxnreg): the two control warpgroups (MMA issuers, loaders)
 // drop to kCtrlRegs, the softmax warpgroups rise to kSoftRegs. The sum must not
@@ -73,6 +79,7 @@ constexpr int kCtrlRegs = 48, kSoftRegs = 96;
 constexpr int kRegsNeeded = 2 * NSLOT * 32 * kCtrlRegs + 4 * NSLOT * 32 * kSoftRegs;
 constexpr uint32_t TMEM_COLS = 512;         // 128 columns per slot
 constexpr float kRescaleLog2 = 8.0f;        // lazy rescale threshold (factor 256)
+constexpr int kMaxMirrors = 7;              // output copies beyond `out` (8 ranks of one node)
 
 // Tensor-memory map of a slot (128 columns). An M=64 accumulator occupies 16
 // of the 32 lanes of each sub-partition (row r in lane 32*(r/16) + r%16 + base,
@@ -121,9 +128,19 @@ struct TcParams {
     const float *o_cg;      // [slabs*m][64]
     __nv_bfloat16 *out;     // [slabs*N][64]
     uint32_t *status;       // nullable
+    // training outputs (all null, or all set): the normalised branch outputs and the
+    // log-sum-exp (natural log) of each row's scaled logits per branch, for the backward
+    __nv_bfloat16 *o_fg, *o_l;   // [slabs*N][64]
+    float *lse;                  // [slabs*N][2]: (FG, L)
+    // further buffers that receive every output row at the same offset as `out` (the
+    // sharded forward's all-gather done by the epilogue's stores, e.g. into peers' memory)
+    __nv_bfloat16 *mirror[kMaxMirrors];
+    int n_mirror;
     int64_t n_tokens;
-    int64_t total_blocks;   // slabs * m query blocks
-    int m, n, w;
+    int64_t total_blocks;   // slabs * tiles query tiles (64 rows each)
+    int64_t tiles;          // 64-row tiles per slab (N / 64)
+    int m, n, w;            // blocks per slab, top-n, window (in blocks)
+    int R;                  // 64-row tiles per block (block_size / 64)
     float scale_log2;
     int64_t withhold_v_step;   // test hook, -1 = off
 };
@@ -194,6 +211,37 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return r;
 }
 
+// 2^x for a pair of fp32 values on the FMA pipe: Cody-Waite split x = n + f with
+// n = round(x) (the 1.5·2^23 shift rounds to nearest in the low mantissa bits) and
+// f in [-1/2, 1/2], 2^f from the degree-3 minimax polynomial of relative error
+// 7.5e-5 (Remez exchange; exp2_fit.py gives the coefficients), and 2^n added to
+// the exponent field. x is clamped at -125, so that the exponent field stays
+// positive (smaller inputs give about 2^-125 instead of 0, immaterial next to a
+// softmax row sum of at least 1); the kernel's x never exceeds the lazy-rescale
+// threshold (2^8), far from overflow.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 shift = make_float2(0x1.8p23f, 0x1.8p23f);
+    const float2 t = __fadd2_rn(x, shift);                         // low bits: round(x)
+    const float2 n = __fadd2_rn(t, make_float2(-0x1.8p23f, -0x1.8p23f));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);   // x - n, exact
+    float2 p = __ffma2_rn(f, make_float2(0x1.c3f76p-5f, 0x1.c3f76p-5f), make_float2(0x1.f0de1ap-3f, 0x1.f0de1ap-3f));
+    p = __ffma2_rn(p, f, make_float2(0x1.62f31ap-1f, 0x1.62f31ap-1f));
+    p = __ffma2_rn(p, f, make_float2(0x1.fff692p-1f, 0x1.fff692p-1f));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// 32 consecutive values x[e]·f as bf16 at dst (64 B, 16-byte aligned).
+__device__ __forceinline__ void store_row32(__nv_bfloat16 *dst, const float *x, float f) {
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        d4[c] = make_uint4(pack_bf16(x[8 * c] * f, x[8 * c + 1] * f), pack_bf16(x[8 * c + 2] * f, x[8 * c + 3] * f),
+                           pack_bf16(x[8 * c + 4] * f, x[8 * c + 5] * f), pack_bf16(x[8 * c + 6] * f, x[8 * c + 7] * f));
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 descriptor version.
 __device__ __forceinline__ uint64_t smem_desc(const void *tile, uint32_t lbo_bytes, uint32_t sbo_bytes) {
     const uint32_t a = smem_u32(tile);
@@ -225,7 +273,7 @@ constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);
 __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUtensorMap *tk,
                             const CUtensorMap *tv, SlotTiles &S, SlotBars &B, int slot,
                             volatile int *abort_flag) {
-    const int L = 2 * p.w + 1, T = L + p.n;
+    const int R = p.R, NR = p.n * R, T = (2 * p.w + 1 + p.n) * R;
     const int64_t stride = NSLOT * (int64_t)gridDim.x;
     uint32_t c = 0, gk = 0, gv = 0;
     uint64_t *last_bar[3] = {nullptr, nullptr, nullptr};   // Q, K, V: most recent copy
@@ -236,35 +284,39 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
         return __all_sync(0xffffffffu, wait_fast(b, par, abort_flag, p.status));
     };
     for (int64_t qi = NSLOT * (int64_t)blockIdx.x + slot; qi < p.total_blocks && ok; qi += stride, ++c) {
-        const int64_t slab = qi / p.m;
-        const int i = (int)(qi - slab * p.m);
+        const int64_t slab = qi / p.tiles;
+        const int qt = (int)(qi - slab * p.tiles), i = qt / R;   // query tile and its block
         const int64_t base = slab * p.n_tokens;
-        const int32_t *ix = p.idx + qi * (int64_t)p.n;
-        auto block_of = [&](int t, int jsel) -> int {
-            const int j = t < p.n ? jsel : i - p.w + (t - p.n);
-            return (j >= 0 && j < p.m) ? j : i;
+        const int32_t *ix = p.idx + (slab * p.m + i) * (int64_t)p.n;
+        // key tile of step t: tile t%R of the (t/R)-th selected block, then of window block
+        // i-w+(t-nR)/R; blocks outside [0, m) are loaded as the query tile and masked
+        auto tile_of = [&](int t, int jsel) -> int {
+            const int j = t < NR ? jsel : i - p.w + (t - NR) / R;
+            return (j >= 0 && j < p.m) ? j * R + t % R : qt;
         };
-        int jq[3];                          // selected indices of steps t, t+1, t+2 (ring)
-        jq[0] = p.n > 0 ? __ldg(ix) : 0;
-        jq[1] = p.n > 1 ? __ldg(ix + 1) : 0;
-        jq[2] = p.n > 2 ? __ldg(ix + 2) : 0;
+        auto sel_at = [&](int u) -> int { return u < NR ? __ldg(ix + u / R) : 0; };
+        int jq[3];                          // selected blocks of steps t, t+1, t+2 (ring)
+        jq[0] = sel_at(0);
+        jq[1] = sel_at(1);
+        jq[2] = sel_at(2);
         // Q of this query block (single buffer: freed by the previous block's last S)
         if (!(ok = wait_w(&B.q_empty, (c & 1) ^ 1))) break;
         if (leader) {
             mbar_expect_tx(&B.q_full, TILE);
-            tma_load_tile(S.q, tq, &B.q_full, (int)(base + (int64_t)i * BK));
+            tma_load_tile(S.q, tq, &B.q_full, (int)(base + (int64_t)qt * BK));
         }
         __syncwarp();
         last_bar[0] = &B.q_full;
         last_par[0] = c & 1;
         int jv = 0;                         // block of the next V copy
         auto issue_k = [&](int t, int j) -> bool {
-            if (leader && t < p.n && (j < 0 || j >= p.m) && p.status) atomicOr(p.status, kStatusBadIndex);
+            if (leader && t < NR && t % R == 0 && (j < 0 || j >= p.m) && p.status)
+                atomicOr(p.status, kStatusBadIndex);
             const int st = gk % NSTAGE;
             if (!wait_w(&B.k_empty[st], ((gk / NSTAGE) & 1) ^ 1)) return false;
             if (leader) {
                 mbar_expect_tx(&B.k_full[st], TILE);
-                tma_load_tile(S.k[st], tk, &B.k_full[st], (int)(base + (int64_t)block_of(t, j) * BK));
+                tma_load_tile(S.k[st], tk, &B.k_full[st], (int)(base + (int64_t)tile_of(t, j) * BK));
             }
             __syncwarp();
             last_bar[1] = &B.k_full[st];
@@ -278,7 +330,7 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
             if (!((int64_t)gv == p.withhold_v_step && blockIdx.x == 0 && slot == 0)) {   // test hook
                 if (leader) {
                     mbar_expect_tx(&B.v_full[st], TILE);
-                    tma_load_tile(S.v[st], tv, &B.v_full[st], (int)(base + (int64_t)block_of(t, j) * BK));
+                    tma_load_tile(S.v[st], tv, &B.v_full[st], (int)(base + (int64_t)tile_of(t, j) * BK));
                 }
                 __syncwarp();
                 last_bar[2] = &B.v_full[st];
@@ -291,8 +343,7 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
         jv = jq[0];
         for (int t = 0; t < T; ++t) {
             const int jk = jq[(t + 1) % 3];   // index of step t+1
-            if (t + 3 < p.n) jq[(t + 3) % 3] = __ldg(ix + t + 3);
-            else jq[(t + 3) % 3] = jq[t % 3];
+            jq[(t + 3) % 3] = t + 3 < NR ? sel_at(t + 3) : jq[t % 3];
             // (the slot just refilled held step t's index, already used by K(t) and kept in jv)
             if (t + 1 < T && !(ok = issue_k(t + 1, jk))) break;
             if (!(ok = issue_v(t, jv))) break;
@@ -307,7 +358,7 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
 
 __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t tmem_slot, int slot,
                          volatile int *abort_flag) {
-    const int L = 2 * p.w + 1, T = L + p.n;
+    const int NR = p.n * p.R, T = (2 * p.w + 1 + p.n) * p.R;
     const int64_t stride = NSLOT * (int64_t)gridDim.x;
     const uint32_t tS = tmem_slot + S_COL + (S_LANE << 16), tO = tmem_slot + O_COL + (O_LANE << 16);
     const uint32_t tP = tmem_slot + P_COL + (P_LANE << 16);   // P buffer b at + 32*b (P in TMEM)
@@ -350,7 +401,7 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
             if (!(ok = wait_w(&B.p_full[pb], (g >> 1) & 1))) break;
             if (!(ok = wait_w(&B.v_full[vs], (g / NSTAGE) & 1))) break;
             fence_after();
-            const uint32_t acc0 = (t == 0 || t == p.n) ? 0u : 1u;   // each branch starts a fresh O
+            const uint32_t acc0 = (t == 0 || t == NR) ? 0u : 1u;   // each branch starts a fresh O
             const uint64_t dv = dv0 + (uint64_t)(vs * (TILE >> 4));
             const uint64_t dp = pb ? dp1 : dp0;
             if (leader) {
@@ -381,7 +432,7 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
 __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t tmem_slot, int slot,
                              int wq, int lane, volatile int *abort_flag) {
     const unsigned FULL = 0xffffffffu;
-    const int L = 2 * p.w + 1, T = L + p.n;
+    const int R = p.R, NR = p.n * R, T = (2 * p.w + 1 + p.n) * R;
     const int ch = lane >> 4;              // column half of the row
     const int r = 16 * wq + (lane & 15);   // row within the query block
     const uint32_t wl = (uint32_t)(32 * wq);   // this warp's sub-partition
@@ -399,22 +450,27 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
         const bool mine = wait_fast(b, par, abort_flag, p.status);
         return __all_sync(FULL, mine);
     };
-    int j0 = 0, j1 = 0;                    // this lane's two selected indices of the next query block
+    // selected blocks of query tile q (its block's index row)
+    auto sel_row = [&](int64_t q) -> const int32_t * {
+        const int64_t sl = q / p.tiles;
+        return p.idx + (sl * p.m + (q - sl * p.tiles) / R) * (int64_t)p.n;
+    };
+    int j0 = 0, j1 = 0;                    // this lane's two selected indices of the next query tile
     {
         const int64_t q0 = NSLOT * (int64_t)blockIdx.x + slot;
         if (q0 < p.total_blocks) {
-            const int32_t *ix = p.idx + q0 * (int64_t)p.n;
+            const int32_t *ix = sel_row(q0);
             if (lane < p.n) j0 = __ldg(ix + lane);
             if (lane + 32 < p.n) j1 = __ldg(ix + lane + 32);
         }
     }
     for (int64_t qi = NSLOT * (int64_t)blockIdx.x + slot; qi < p.total_blocks && ok; qi += stride) {
-        const int64_t slab = qi / p.m;
-        const int i = (int)(qi - slab * p.m);
-        const int64_t tok = slab * p.n_tokens + (int64_t)i * BK + r;
+        const int64_t slab = qi / p.tiles;
+        const int qt = (int)(qi - slab * p.tiles), i = qt / R;   // query tile and its block
+        const int64_t tok = slab * p.n_tokens + (int64_t)qt * BK + r;
         const float *gp = p.gates + tok * 3;
         const float g_cg = __ldg(gp), g_fg = __ldg(gp + 1), g_l = __ldg(gp + 2);
-        const float *ocg = p.o_cg + qi * (int64_t)HD + 32 * ch;
+        const float *ocg = p.o_cg + (slab * p.m + i) * (int64_t)HD + 32 * ch;
         asm volatile("prefetch.global.L1 [%0];" ::"l"(ocg));
         // validity of the n selected blocks of this query block, as a bit mask
         // (its indices were fetched during the previous query block)
@@ -425,22 +481,23 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             const int64_t qn = qi + stride;
             j0 = j1 = 0;
             if (qn < p.total_blocks) {
-                const int32_t *ix = p.idx + qn * (int64_t)p.n;
+                const int32_t *ix = sel_row(qn);
                 if (lane < p.n) j0 = __ldg(ix + lane);
                 if (lane + 32 < p.n) j1 = __ldg(ix + lane + 32);
             }
         }
-        float m_used = -INFINITY, l_run = 0.f, l_sel = 0.f;
+        float m_used = -INFINITY, l_run = 0.f, l_sel = 0.f, m_sel = -INFINITY;
         for (int t = 0; t < T; ++t, ++g) {
             bool valid;
-            if (t < p.n) {
-                valid = (selmask >> t) & 1u;
+            if (t < NR) {
+                valid = (selmask >> (t / R)) & 1u;
             } else {
-                const int j = i - p.w + (t - p.n);
+                const int j = i - p.w + (t - NR) / R;
                 valid = j >= 0 && j < p.m;
             }
-            if (t == p.n) {                    // the local branch starts afresh
+            if (t == NR) {                     // the local branch starts afresh
                 l_sel = l_run;
+                m_sel = m_used;
                 l_run = 0.f;
                 m_used = -INFINITY;
             }
@@ -468,7 +525,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
                     const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
-                    const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                    const float2 e = (c < POLY_PAIRS) ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
                     pk[c] = pack_bf16(e.x, e.y);
                     acc2[c & 1] = __fadd2_rn(acc2[c & 1], e);
                 }
@@ -482,10 +539,10 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             //      must be complete
             // (S(g) complete implies P·V(g-2) complete: one thread issues both, in order,
             //  so the two-barrier parity below cannot alias)
-            const bool touch_o = (t == p.n) || __any_sync(FULL, need);
+            const bool touch_o = (t == NR) || __any_sync(FULL, need);
             if (touch_o && g > 0 && !(ok = wait_all(&B.o_done[(g - 1) & 1], ((g - 1) >> 1) & 1))) break;
             fence_after();
-            if (t == p.n) {
+            if (t == NR) {
                 // close the selection branch: acc = g_CG·o_CG + g_FG·o_FG, kept in fp32 in
                 // this row's lanes of the other lane half until the epilogue
                 const float l = l_sel + __shfl_xor_sync(FULL, l_sel, 16);
@@ -494,6 +551,11 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 tmem_ld16(tO, a);
                 tmem_ld16(tO + 16, a + 16);
                 tmem_wait_ld();
+                if (p.o_fg) {                  // training: o_FG and its row log-sum-exp
+                    const float inv1 = l > 0.f ? 1.f / l : 0.f;
+                    store_row32(p.o_fg + tok * HD + 32 * ch, a, inv1);
+                    if (ch == 0) p.lse[tok * 2] = (m_sel + __log2f(l)) * 0.69314718055994531f;
+                }
 #pragma unroll
                 for (int e = 0; e < 32; ++e) a[e] = fmaf(g_cg, __ldg(ocg + e), a[e] * inv);
                 tmem_st16(tA, a);
@@ -542,6 +604,14 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
         fence_after();
         const float l = l_run + __shfl_xor_sync(FULL, l_run, 16);
         const float inv = l > 0.f ? g_l / l : 0.f;
+        if (p.o_l) {                           // training: o_L and its row log-sum-exp
+            float o[32];
+            tmem_ld16(tO, o);
+            tmem_ld16(tO + 16, o + 16);
+            tmem_wait_ld();
+            store_row32(p.o_l + tok * HD + 32 * ch, o, l > 0.f ? 1.f / l : 0.f);
+            if (ch == 0) p.lse[tok * 2 + 1] = (m_used + __log2f(l)) * 0.69314718055994531f;
+        }
         uint4 *d4 = reinterpret_cast<uint4 *>(p.out + tok * HD + 32 * ch);
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
@@ -553,8 +623,14 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
 #pragma unroll
             for (int e = 0; e < 8; ++e)
                 w8[e] = pack_bf16(fmaf(o[2 * e], inv, a[2 * e]), fmaf(o[2 * e + 1], inv, a[2 * e + 1]));
-            d4[2 * cc] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-            d4[2 * cc + 1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+            const uint4 lo4 = make_uint4(w8[0], w8[1], w8[2], w8[3]), hi4 = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+            d4[2 * cc] = lo4;
+            d4[2 * cc + 1] = hi4;
+            for (int mi = 0; mi < p.n_mirror; ++mi) {
+                uint4 *m4 = reinterpret_cast<uint4 *>(p.mirror[mi] + tok * HD + 32 * ch);
+                m4[2 * cc] = lo4;
+                m4[2 * cc + 1] = hi4;
+            }
         }
         fence_before();
     }
@@ -631,44 +707,35 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
 
 // --------------------------------------------------------------- host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
 bool make_tile_map(CUtensorMap *map, const void *base, uint64_t rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)HD, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)HD * 2};
-    cuuint32_t box[2] = {(cuuint32_t)HD, (cuuint32_t)BK};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return make_tile_map_bf16x64(map, base, rows);
 }
 
-int sm_count() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    return n;
+// Test hook: y = exp2_poly2(x) (poly != 0) or ex2.approx(x), elementwise.
+__global__ void exp2_eval_kernel(const float *__restrict__ x, float *__restrict__ y, int64_t n, int poly) {
+    for (int64_t i = 2 * (blockIdx.x * (int64_t)blockDim.x + threadIdx.x); i < n;
+         i += 2 * (int64_t)gridDim.x * blockDim.x) {
+        const float2 v = make_float2(x[i], i + 1 < n ? x[i + 1] : 0.f);
+        const float2 e = poly ? exp2_poly2(v) : make_float2(ex2(v.x), ex2(v.y));
+        y[i] = e.x;
+        if (i + 1 < n) y[i + 1] = e.y;
+    }
 }
 
 }  // namespace
 
+cudaError_t launch_exp2_eval(const float *x, float *y, int64_t n, int poly, cudaStream_t stream) {
+    int64_t ctas = (n / 2 + 255) / 256 + 1;
+    if (ctas > 148 * 16) ctas = 148 * 16;
+    exp2_eval_kernel<<<(unsigned)ctas, 256, 0, stream>>>(x, y, n, poly);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_attend_tc(const Problem &pb, const void *q, const void *k, const void *v,
                              const float *gates, const float *o_cg, const int32_t *idx, void *out,
-                             uint32_t *status, cudaStream_t stream) {
-    if (pb.dtype != BSA_BF16 || pb.block_size != BK || pb.head_dim != HD) return cudaErrorNotSupported;
+                             uint32_t *status, cudaStream_t stream, void *o_fg, void *o_l, float *lse,
+                             void *const *mirrors, int n_mirrors) {
+    if (pb.dtype != BSA_BF16 || pb.block_size % BK != 0 || pb.head_dim != HD) return cudaErrorNotSupported;
     const int64_t rows = pb.slabs * pb.n_tokens;
     if (rows > 0x7fffffffLL) return cudaErrorNotSupported;       // TMA row coordinate is int32
     CUtensorMap tq, tk, tv;
@@ -680,11 +747,20 @@ cudaError_t launch_attend_tc(const Problem &pb, const void *q, const void *k, co
     p.o_cg = o_cg;
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.status = status;
+    p.o_fg = static_cast<__nv_bfloat16 *>(o_fg);
+    p.o_l = static_cast<__nv_bfloat16 *>(o_l);
+    p.lse = lse;
+    if ((o_fg || o_l || lse) && !(o_fg && o_l && lse)) return cudaErrorInvalidValue;
+    if (n_mirrors < 0 || n_mirrors > kMaxMirrors || (n_mirrors > 0 && !mirrors)) return cudaErrorInvalidValue;
+    p.n_mirror = n_mirrors;
+    for (int i = 0; i < kMaxMirrors; ++i) p.mirror[i] = i < n_mirrors ? static_cast<__nv_bfloat16 *>(mirrors[i]) : nullptr;
     p.n_tokens = pb.n_tokens;
     p.m = (int)pb.m;
     p.n = (int)pb.top_n;
     p.w = (int)pb.window;
-    p.total_blocks = pb.slabs * pb.m;
+    p.R = (int)(pb.block_size / BK);
+    p.tiles = pb.n_tokens / BK;
+    p.total_blocks = pb.slabs * p.tiles;
     p.scale_log2 = pb.scale * 1.4426950408889634f;
     p.withhold_v_step = pb.withhold_v_step;
     const int sms = sm_count();

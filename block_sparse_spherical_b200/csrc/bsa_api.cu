@@ -16,9 +16,11 @@ size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// bf16: blocks of 64, 256 or 1024 tokens (a parent pixel 3, 4 or 5 levels up), head_dim 64, on
+// the tensor cores; fp32: (16, 32) and (64, 64) on the CUDA cores.
 bool shape_supported(int32_t dtype, int32_t bk, int32_t d) {
-    return (dtype == BSA_BF16 && bk == 64 && d == 64) || (dtype == BSA_F32 && bk == 64 && d == 64) ||
-           (dtype == BSA_F32 && bk == 16 && d == 32);
+    return (dtype == BSA_BF16 && (bk == 64 || bk == 256 || bk == 1024) && d == 64) ||
+           (dtype == BSA_F32 && bk == 64 && d == 64) || (dtype == BSA_F32 && bk == 16 && d == 32);
 }
 
 bsa_status make_problem(const bsa_config *cfg, Problem *p) {
@@ -189,6 +191,230 @@ bsa_status bsa_forward(const bsa_config *cfg, const void *q, const void *k, cons
     void *images = L.total > L.split ? ws + L.split : nullptr;
     if (e == cudaSuccess) e = launch_compress(p, qbar, kbar, vbar, ocg, idx, status, images, stream);
     if (e == cudaSuccess) e = launch_fine(p, q, k, v, gates, ocg, idx, out, status, stream);
+    return from_cuda(e);
+}
+
+// ---- training: forward with saved tensors, and the backward ---------------
+
+namespace {
+
+bool train_supported(const Problem &p) { return p.dtype == BSA_BF16 && p.head_dim == 64; }
+
+struct BwdLayout {
+    size_t status, qbar, kbar, vbar, dfine, docg16, q16, k16, v16, dcg, lse_pad, dqbar, dkbar, dvbar, dq_acc;
+    size_t count, offs, cursor, list_tmp, list, total;
+    int64_t m_pad;
+};
+
+BwdLayout bwd_layout_of(const Problem &p) {
+    BwdLayout L;
+    L.m_pad = (p.m + 63) / 64 * 64;
+    const size_t pooled = (size_t)p.slabs * p.m * p.head_dim * sizeof(float);
+    const size_t pad16 = (size_t)p.slabs * L.m_pad * p.head_dim * 2, pad32 = 2 * pad16;
+    const size_t pad1 = (size_t)p.slabs * L.m_pad * sizeof(float);
+    const size_t rows = (size_t)p.slabs * p.n_tokens;
+    const size_t ints_m = (size_t)p.slabs * p.m * sizeof(int), ints_list = ints_m * p.top_n;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { const size_t at = o; o += round_up(bytes); return at; };
+    L.status = take(kAlign);
+    L.qbar = take(pooled);
+    L.kbar = take(pooled);
+    L.vbar = take(pooled);
+    L.dfine = take(rows * 2 * sizeof(float));
+    L.docg16 = take(pad16);
+    L.q16 = take(pad16);
+    L.k16 = take(pad16);
+    L.v16 = take(pad16);
+    L.dcg = take(pad1);
+    L.lse_pad = take(pad1);
+    L.dqbar = take(pad32);
+    L.dkbar = take(pad32);
+    L.dvbar = take(pad32);
+    L.dq_acc = take(rows * p.head_dim * sizeof(float));
+    L.count = take(ints_m);
+    L.offs = take((size_t)p.slabs * (p.m + 1) * sizeof(int));
+    L.cursor = take(ints_m);
+    L.list_tmp = take(ints_list);
+    L.list = take(ints_list);
+    L.total = o;
+    return L;
+}
+
+}  // namespace
+
+bsa_status bsa_forward_train(const bsa_config *cfg, const void *q, const void *k, const void *v,
+                             const float *gates, void *out, int32_t *sel_idx, float *o_cg_block, float *lse_cg,
+                             void *o_fg, void *o_l, float *lse_fine, void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (!train_supported(p)) return BSA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !gates || !out || !sel_idx || !o_cg_block || !lse_cg || !o_fg || !o_l || !lse_fine)
+        return BSA_ERR_INVALID_ARG;
+    if (!workspace) return BSA_ERR_WORKSPACE;
+    const WorkspaceLayout L = layout_of(p);
+    if (workspace_bytes < L.total) return BSA_ERR_WORKSPACE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gates) || !aligned16(out) ||
+        !aligned16(sel_idx) || !aligned16(o_cg_block) || !aligned16(lse_cg) || !aligned16(o_fg) ||
+        !aligned16(o_l) || !aligned16(lse_fine) || ((uintptr_t)workspace & (kAlign - 1)))
+        return BSA_ERR_ALIGNMENT;
+    char *ws = static_cast<char *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws + L.status);
+    float *qbar = reinterpret_cast<float *>(ws + L.qbar);
+    float *kbar = reinterpret_cast<float *>(ws + L.kbar);
+    float *vbar = reinterpret_cast<float *>(ws + L.vbar);
+    void *images = L.total > L.split ? ws + L.split : nullptr;
+    cudaError_t e = bsa::launch_pool(p, q, k, v, qbar, kbar, vbar, stream);
+    if (e == cudaSuccess) {
+        e = bsa::launch_compress_tc(p, qbar, kbar, vbar, o_cg_block, sel_idx, status, images, stream, lse_cg);
+        if (e == cudaErrorNotSupported)
+            e = bsa::launch_compress_select(p, qbar, kbar, vbar, o_cg_block, sel_idx, stream, lse_cg);
+    }
+    if (e == cudaSuccess)
+        e = bsa::launch_attend_tc(p, q, k, v, gates, o_cg_block, sel_idx, out, status, stream, o_fg, o_l, lse_fine);
+    return from_cuda(e);
+}
+
+bsa_status bsa_backward_workspace_size(const bsa_config *cfg, size_t *bytes) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (!train_supported(p)) return BSA_ERR_UNSUPPORTED;
+    if (!bytes) return BSA_ERR_INVALID_ARG;
+    *bytes = bwd_layout_of(p).total;
+    return BSA_OK;
+}
+
+bsa_status bsa_backward(const bsa_config *cfg, const void *q, const void *k, const void *v, const float *gates,
+                        const void *dout, const int32_t *sel_idx, const float *o_cg_block, const float *lse_cg,
+                        const void *o_fg, const void *o_l, const float *lse_fine, void *dq, void *dk, void *dv,
+                        float *dgates, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (!train_supported(p)) return BSA_ERR_UNSUPPORTED;
+    const void *in[] = {q, k, v, gates, dout, sel_idx, o_cg_block, lse_cg, o_fg, o_l, lse_fine, dq, dk, dv, dgates};
+    for (const void *x : in)
+        if (!x) return BSA_ERR_INVALID_ARG;
+    if (!workspace) return BSA_ERR_WORKSPACE;
+    const BwdLayout L = bwd_layout_of(p);
+    if (workspace_bytes < L.total) return BSA_ERR_WORKSPACE;
+    for (const void *x : in)
+        if (!aligned16(x)) return BSA_ERR_ALIGNMENT;
+    if ((uintptr_t)workspace & (kAlign - 1)) return BSA_ERR_ALIGNMENT;
+    char *ws = static_cast<char *>(workspace);
+    bsa::BwdBuffers b;
+    b.q = q; b.k = k; b.v = v; b.dout = dout; b.gates = gates; b.sel_idx = sel_idx;
+    b.o_cg = o_cg_block; b.lse_cg = lse_cg; b.o_fg = o_fg; b.o_l = o_l; b.lse_fine = lse_fine;
+    b.dq = dq; b.dk = dk; b.dv = dv; b.dgates = dgates;
+    b.m_pad = L.m_pad;
+    b.status = reinterpret_cast<uint32_t *>(ws + L.status);
+    b.qbar = reinterpret_cast<float *>(ws + L.qbar);
+    b.kbar = reinterpret_cast<float *>(ws + L.kbar);
+    b.vbar = reinterpret_cast<float *>(ws + L.vbar);
+    b.dfine = reinterpret_cast<float *>(ws + L.dfine);
+    b.docg16 = ws + L.docg16;
+    b.q16 = ws + L.q16;
+    b.k16 = ws + L.k16;
+    b.v16 = ws + L.v16;
+    b.dcg = reinterpret_cast<float *>(ws + L.dcg);
+    b.lse_cg_pad = reinterpret_cast<float *>(ws + L.lse_pad);
+    b.dqbar = reinterpret_cast<float *>(ws + L.dqbar);
+    b.dkbar = reinterpret_cast<float *>(ws + L.dkbar);
+    b.dvbar = reinterpret_cast<float *>(ws + L.dvbar);
+    b.dq_acc = reinterpret_cast<float *>(ws + L.dq_acc);
+    b.count = reinterpret_cast<int *>(ws + L.count);
+    b.offs = reinterpret_cast<int *>(ws + L.offs);
+    b.cursor = reinterpret_cast<int *>(ws + L.cursor);
+    b.list_tmp = reinterpret_cast<int *>(ws + L.list_tmp);
+    b.list = reinterpret_cast<int *>(ws + L.list);
+    // the two gradient accumulators start at zero (memsets, not allocations)
+    cudaError_t e = cudaMemsetAsync(ws + L.dq_acc, 0, (size_t)p.slabs * p.n_tokens * p.head_dim * sizeof(float),
+                                    stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.dqbar, 0, (size_t)p.slabs * L.m_pad * p.head_dim * 4, stream);
+    if (e == cudaSuccess) e = bsa::launch_pool(p, q, k, v, b.qbar, b.kbar, b.vbar, stream);
+    if (e == cudaSuccess) e = bsa::launch_bwd_prep(p, b, stream);
+    if (e == cudaSuccess) e = bsa::launch_attend_bwd_compressed(p, b, stream);
+    if (e == cudaSuccess)
+        e = bsa::launch_inverse_index(p, sel_idx, b.count, b.offs, b.cursor, b.list_tmp, b.list, b.status, stream);
+    if (e == cudaSuccess) e = bsa::launch_attend_bwd_fine(p, b, stream);
+    if (e == cudaSuccess) e = bsa::launch_bwd_finalize_dq(p, b.dq_acc, b.dqbar, L.m_pad, dq, stream);
+    return from_cuda(e);
+}
+
+bsa_status bsa_permute_tokens(int64_t slabs, int64_t n_tokens, int64_t row_bytes, const int32_t *perm,
+                              const void *src, void *dst, uint32_t *status_word, cudaStream_t stream) {
+    if (slabs < 1 || n_tokens < 1 || n_tokens > 0x7fffffffLL || row_bytes < 4 || row_bytes % 4 != 0 ||
+        row_bytes / 4 > 0x7fffffffLL)
+        return BSA_ERR_INVALID_ARG;
+    if (!perm || !src || !dst) return BSA_ERR_INVALID_ARG;
+    if (src == dst) return BSA_ERR_INVALID_ARG;        // rows move between two distinct buffers
+    const uintptr_t need = row_bytes % 16 == 0 ? 15u : 3u;
+    if (((uintptr_t)src & need) || ((uintptr_t)dst & need) || ((uintptr_t)perm & 3u) || ((uintptr_t)status_word & 3u))
+        return BSA_ERR_ALIGNMENT;
+    return from_cuda(bsa::launch_permute_rows(src, dst, perm, slabs, n_tokens, row_bytes, status_word, stream));
+}
+
+bsa_status bsa_latlon_healpix_plan(int64_t nside, int64_t nlat, int64_t nlon, int32_t *nbr, float *rel,
+                                   cudaStream_t stream) {
+    if (nside < 1 || nside > (1 << 13) || (nside & (nside - 1)) || nlat < 4 || nlon < 4 ||
+        (int64_t)nlat * nlon > 0x7fffffffLL)
+        return BSA_ERR_INVALID_ARG;
+    if (!nbr || !rel) return BSA_ERR_INVALID_ARG;
+    if (((uintptr_t)nbr & 15u) || ((uintptr_t)rel & 15u)) return BSA_ERR_ALIGNMENT;
+    return from_cuda(bsa::launch_healpix_plan(nside, nlat, nlon, nbr, rel, stream));
+}
+
+bsa_status bsa_latlon_to_healpix(int64_t batch, int64_t n_tgt, int64_t n_src, int64_t head_dim, int32_t dtype,
+                                 float scale, const int32_t *nbr, const float *rel, const float *wq,
+                                 const void *k_src, const void *v_src, void *out, uint32_t *status_word,
+                                 cudaStream_t stream) {
+    if (batch < 1 || batch > 65535 || n_tgt < 1 || n_src < 1 || n_src > 0x7fffffffLL) return BSA_ERR_INVALID_ARG;
+    if (dtype != BSA_F32 && dtype != BSA_BF16) return BSA_ERR_INVALID_ARG;
+    if (!(scale >= 0.0f) || isinf(scale)) return BSA_ERR_INVALID_ARG;
+    if (head_dim != 32 && head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
+    if (!nbr || !rel || !wq || !k_src || !v_src || !out) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(nbr) || !aligned16(rel) || !aligned16(wq) || !aligned16(k_src) || !aligned16(v_src) ||
+        !aligned16(out) || ((uintptr_t)status_word & 3u))
+        return BSA_ERR_ALIGNMENT;
+    const float s = scale > 0.0f ? scale : 1.0f / sqrtf((float)head_dim);
+    return from_cuda(bsa::launch_interp(batch, n_tgt, n_src, head_dim, (bsa_dtype)dtype, nbr, rel, wq, k_src, v_src,
+                                        out, s, status_word, stream));
+}
+
+bsa_status bsa_forward_mirrored(const bsa_config *cfg, const void *q, const void *k, const void *v,
+                                const float *gates, void *out, void *const *mirrors, int32_t n_mirrors,
+                                int32_t *sel_idx_out, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    Problem p;
+    bsa_status st = make_problem(cfg, &p);
+    if (st != BSA_OK) return st;
+    if (p.dtype != BSA_BF16) return BSA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !gates || !out || n_mirrors < 0 || n_mirrors > 7 || (n_mirrors > 0 && !mirrors))
+        return BSA_ERR_INVALID_ARG;
+    for (int i = 0; i < n_mirrors; ++i) {
+        if (!mirrors[i] || mirrors[i] == out) return BSA_ERR_INVALID_ARG;
+        if (!aligned16(mirrors[i])) return BSA_ERR_ALIGNMENT;
+    }
+    if (!workspace) return BSA_ERR_WORKSPACE;
+    const WorkspaceLayout L = layout_of(p);
+    if (workspace_bytes < L.total) return BSA_ERR_WORKSPACE;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gates) || !aligned16(out) ||
+        !aligned16(sel_idx_out) || ((uintptr_t)workspace & (kAlign - 1)))
+        return BSA_ERR_ALIGNMENT;
+    char *ws = static_cast<char *>(workspace);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws + L.status);
+    float *qbar = reinterpret_cast<float *>(ws + L.qbar);
+    float *kbar = reinterpret_cast<float *>(ws + L.kbar);
+    float *vbar = reinterpret_cast<float *>(ws + L.vbar);
+    float *ocg = reinterpret_cast<float *>(ws + L.o_cg);
+    int32_t *idx = sel_idx_out ? sel_idx_out : reinterpret_cast<int32_t *>(ws + L.idx);
+    void *images = L.total > L.split ? ws + L.split : nullptr;
+    cudaError_t e = bsa::launch_pool(p, q, k, v, qbar, kbar, vbar, stream);
+    if (e == cudaSuccess) e = launch_compress(p, qbar, kbar, vbar, ocg, idx, status, images, stream);
+    if (e == cudaSuccess)
+        e = bsa::launch_attend_tc(p, q, k, v, gates, ocg, idx, out, status, stream, nullptr, nullptr, nullptr, mirrors,
+                                  n_mirrors);
     return from_cuda(e);
 }
 
@@ -373,4 +599,12 @@ extern "C" bsa_status bsa_testing_fine_attention_withhold(const bsa_config *cfg,
     if (withhold_v_step < 0) return BSA_ERR_INVALID_ARG;
     p.withhold_v_step = withhold_v_step;
     return from_cuda(bsa::launch_attend_tc(p, q, k, v, gates, o_cg_block, sel_idx, out, status_word, stream));
+}
+
+// Test hook (include/bsa_testing.h): the softmax's two exp2 routes, elementwise.
+extern "C" bsa_status bsa_testing_exp2(const float *x, float *y, int64_t n, int32_t poly, cudaStream_t stream) {
+    if (!x || !y || n < 0) return BSA_ERR_INVALID_ARG;
+    if (((uintptr_t)x & 3u) || ((uintptr_t)y & 3u)) return BSA_ERR_ALIGNMENT;
+    if (n == 0) return BSA_OK;
+    return from_cuda(bsa::launch_exp2_eval(x, y, n, poly, stream));
 }

@@ -120,7 +120,8 @@ template <int D, int NPL>
 __global__ void __launch_bounds__(256, 2)
 compress_select_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar,
                        const float *__restrict__ vbar, float *__restrict__ o_cg,
-                       int32_t *__restrict__ idx_out, int m, int n, float scale_log2) {
+                       int32_t *__restrict__ idx_out, int m, int n, float scale_log2,
+                       float *__restrict__ lse_out) {
     static_assert(D == 32 || D == 64, "head_dim 32 or 64");
     constexpr int DPT = D / 16;                // output columns per thread
     extern __shared__ __align__(16) float smem[];
@@ -357,6 +358,8 @@ compress_select_kernel(const float *__restrict__ qbar, const float *__restrict__
                 *reinterpret_cast<float4 *>(dst) = make_float4(oi[0], oi[1], oi[2], oi[3]);
             else
                 *reinterpret_cast<float2 *>(dst) = make_float2(oi[0], oi[1]);
+            // training: natural-log log-sum-exp of the row's scaled logits
+            if (lse_out && tx == 0) lse_out[slab * m + r] = (mrun[i] + log2f(l)) * 0.69314718055994531f;
             int32_t *ix = idx_out + (slab * m + r) * (int64_t)n;
 #pragma unroll
             for (int h = 0; h < NPL; ++h) {
@@ -369,14 +372,14 @@ compress_select_kernel(const float *__restrict__ qbar, const float *__restrict__
 
 template <int D, int NPL>
 cudaError_t launch(const Problem &p, const float *qb, const float *kb, const float *vb, float *ocg,
-                   int32_t *idx, cudaStream_t s) {
+                   int32_t *idx, cudaStream_t s, float *lse) {
     const size_t smem = (size_t)(BM * LDS + 4 * BN * LDS + BM * LDS) * sizeof(float);
     auto kern = compress_select_kernel<D, NPL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((p.m + BM - 1) / BM), (unsigned)p.slabs);
     const float scale_log2 = p.scale * 1.4426950408889634f;
-    kern<<<grid, 256, smem, s>>>(qb, kb, vb, ocg, idx, (int)p.m, (int)p.top_n, scale_log2);
+    kern<<<grid, 256, smem, s>>>(qb, kb, vb, ocg, idx, (int)p.m, (int)p.top_n, scale_log2, lse);
     return cudaGetLastError();
 }
 
@@ -384,21 +387,21 @@ cudaError_t launch(const Problem &p, const float *qb, const float *kb, const flo
 
 cudaError_t launch_compress_select(const Problem &p, const float *qbar, const float *kbar,
                                    const float *vbar, float *o_cg, int32_t *idx,
-                                   cudaStream_t stream) {
+                                   cudaStream_t stream, float *lse) {
     if (p.top_n > kMaxTopN) return cudaErrorNotSupported;
     const int npl = (int)((p.top_n + 15) / 16);
     if (p.head_dim == 64) {
         switch (npl) {
-            case 1: return launch<64, 1>(p, qbar, kbar, vbar, o_cg, idx, stream);
-            case 2: return launch<64, 2>(p, qbar, kbar, vbar, o_cg, idx, stream);
-            default: return launch<64, 4>(p, qbar, kbar, vbar, o_cg, idx, stream);
+            case 1: return launch<64, 1>(p, qbar, kbar, vbar, o_cg, idx, stream, lse);
+            case 2: return launch<64, 2>(p, qbar, kbar, vbar, o_cg, idx, stream, lse);
+            default: return launch<64, 4>(p, qbar, kbar, vbar, o_cg, idx, stream, lse);
         }
     }
     if (p.head_dim == 32) {
         switch (npl) {
-            case 1: return launch<32, 1>(p, qbar, kbar, vbar, o_cg, idx, stream);
-            case 2: return launch<32, 2>(p, qbar, kbar, vbar, o_cg, idx, stream);
-            default: return launch<32, 4>(p, qbar, kbar, vbar, o_cg, idx, stream);
+            case 1: return launch<32, 1>(p, qbar, kbar, vbar, o_cg, idx, stream, lse);
+            case 2: return launch<32, 2>(p, qbar, kbar, vbar, o_cg, idx, stream, lse);
+            default: return launch<32, 4>(p, qbar, kbar, vbar, o_cg, idx, stream, lse);
         }
     }
     return cudaErrorNotSupported;

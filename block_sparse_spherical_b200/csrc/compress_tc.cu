@@ -91,6 +91,7 @@ struct Args {
     const uint8_t *qimg, *kimg, *vimg;     // this slab's split images (workspace path), else null
     float *o_cg;                           // this slab's [m][64]
     int32_t *idx;                          // this slab's [m][n]
+    float *lse;                            // this slab's [m] (training output), or null
     int m;
     float sl2;                             // s·log2(e)
     uint32_t *status;                      // nullable
@@ -473,6 +474,8 @@ __device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter
         return;
     }
     const float inv = 1.f / l_run;
+    // training: natural-log log-sum-exp of the row's scaled logits
+    if (a.lse) a.lse[row] = (m_run + log2f(l_run)) * 0.69314718055994531f;
     float4 *dst = reinterpret_cast<float4 *>(a.o_cg + (int64_t)row * D);
 #pragma unroll
     for (int c = 0; c < D / 4; ++c)
@@ -486,7 +489,7 @@ template <int NSEL, bool PRE>
 __global__ void __launch_bounds__(NTHREADS, 1)
 compress_tc_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar, const float *__restrict__ vbar,
                    float *__restrict__ o_cg, int32_t *__restrict__ idx, int m, float sl2, uint32_t *status,
-                   const uint8_t *__restrict__ images) {
+                   const uint8_t *__restrict__ images, float *__restrict__ lse) {
     extern __shared__ uint8_t smem_raw[];
     Smem &sh = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -499,6 +502,7 @@ compress_tc_kernel(const float *__restrict__ qbar, const float *__restrict__ kba
     a.v = vbar + slab * (int64_t)m * D;
     a.o_cg = o_cg + slab * (int64_t)m * D;
     a.idx = idx + slab * (int64_t)m * NSEL;
+    a.lse = lse ? lse + slab * (int64_t)m : nullptr;
     a.m = m;
     a.sl2 = sl2;
     a.status = status;
@@ -622,29 +626,38 @@ split_images_kernel(const float *__restrict__ qbar, const float *__restrict__ kb
     }
 }
 
-template <bool PRE>
-cudaError_t launch_tc(const Problem &p, const float *qbar, const float *kbar, const float *vbar, float *o_cg,
-                      int32_t *idx, uint32_t *status, const uint8_t *images, cudaStream_t stream) {
+template <int NSEL, bool PRE>
+cudaError_t launch_tc_n(const Problem &p, const float *qbar, const float *kbar, const float *vbar, float *o_cg,
+                        int32_t *idx, uint32_t *status, const uint8_t *images, cudaStream_t stream, float *lse) {
     const size_t smem = sizeof(Smem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(compress_tc_kernel<16, PRE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(compress_tc_kernel<NSEL, PRE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     // the register split must fit the registers the CTA is launched with
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, compress_tc_kernel<16, PRE>);
+    e = cudaFuncGetAttributes(&fa, compress_tc_kernel<NSEL, PRE>);
     if (e != cudaSuccess) return e;
     if ((int64_t)fa.numRegs * NTHREADS < kRegsNeeded || fa.maxThreadsPerBlock < NTHREADS)
         return cudaErrorInvalidConfiguration;
     const dim3 grid((unsigned)((p.m + BM - 1) / BM), (unsigned)p.slabs);
-    compress_tc_kernel<16, PRE><<<grid, NTHREADS, smem, stream>>>(qbar, kbar, vbar, o_cg, idx, (int)p.m,
-                                                                   p.scale * 1.4426950408889634f, status, images);
+    compress_tc_kernel<NSEL, PRE><<<grid, NTHREADS, smem, stream>>>(qbar, kbar, vbar, o_cg, idx, (int)p.m,
+                                                                     p.scale * 1.4426950408889634f, status, images,
+                                                                     lse);
     return cudaGetLastError();
+}
+
+template <bool PRE>
+cudaError_t launch_tc(const Problem &p, const float *qbar, const float *kbar, const float *vbar, float *o_cg,
+                      int32_t *idx, uint32_t *status, const uint8_t *images, cudaStream_t stream, float *lse) {
+    if (p.top_n == 32)
+        return launch_tc_n<32, PRE>(p, qbar, kbar, vbar, o_cg, idx, status, images, stream, lse);
+    return launch_tc_n<16, PRE>(p, qbar, kbar, vbar, o_cg, idx, status, images, stream, lse);
 }
 
 }  // namespace
 
 bool compress_tc_supported(const Problem &p) {
-    return p.head_dim == D && p.top_n == 16 && p.m <= 0x7fffffffLL / D;
+    return p.head_dim == D && (p.top_n == 16 || p.top_n == 32) && p.m <= 0x7fffffffLL / D;
 }
 
 size_t compress_tc_workspace_bytes(const Problem &p) {
@@ -654,14 +667,16 @@ size_t compress_tc_workspace_bytes(const Problem &p) {
 }
 
 cudaError_t launch_compress_tc(const Problem &p, const float *qbar, const float *kbar, const float *vbar,
-                               float *o_cg, int32_t *idx, uint32_t *status, void *images, cudaStream_t stream) {
+                               float *o_cg, int32_t *idx, uint32_t *status, void *images, cudaStream_t stream,
+                               float *lse) {
     if (!compress_tc_supported(p)) return cudaErrorNotSupported;
-    if (!images) return launch_tc<false>(p, qbar, kbar, vbar, o_cg, idx, status, nullptr, stream);
+    if (!images) return launch_tc<false>(p, qbar, kbar, vbar, o_cg, idx, status, nullptr, stream, lse);
     const dim3 sgrid((unsigned)((p.m + BM - 1) / BM * 2), (unsigned)p.slabs);
     split_images_kernel<<<sgrid, 256, 0, stream>>>(qbar, kbar, vbar, static_cast<uint8_t *>(images), (int)p.m);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return launch_tc<true>(p, qbar, kbar, vbar, o_cg, idx, status, static_cast<const uint8_t *>(images), stream);
+    return launch_tc<true>(p, qbar, kbar, vbar, o_cg, idx, status, static_cast<const uint8_t *>(images), stream,
+                           lse);
 }
 
 }  // namespace bsa

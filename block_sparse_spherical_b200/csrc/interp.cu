@@ -1,0 +1,192 @@
+// Lat-lon -> HEALPix cross-attention interpolation, the step before BSA in the
+// MOSAIC note's pipeline ("overall framework" (1), HEALPix paragraph): each
+// HEALPix target pixel i attends to its neighbouring source points j of a
+// latitude-longitude grid with the relative position p_ij as the query,
+//   o_i = Σ_{j ∈ N_i} softmax_j((W_q p_ij)·k_j · s) v_j,   s = 1/sqrt(d).
+//
+// healpix_plan_kernel: one thread per NESTED pixel: its centre (the published
+//   HEALPix ring formulas; face from the high bits, in-face (x, y) from the
+//   interleaved low bits), the 4 x 4 block of grid points around it (rows
+//   r0..r0+3, r0 = floor((90 - lat)/dlat) - 1 clamped to [0, nlat-4]; columns
+//   c0-1..c0+2 wrapping in longitude, c0 = floor(lon/dlon)) and the relative
+//   positions (x_j - x_i)/dlat_rad. The integer decisions use fp64.
+// interp_kernel: one warp per target: lane l holds channels l*C..l*C+C-1
+//   (C = d/32); per neighbour the query channels W_q p_ij, a warp-reduced dot
+//   with k_j, then an exact softmax over the 16 logits and the weighted sum
+//   of the v_j rows, which are gathered from the small (L2-resident) source
+//   grid. fp32 arithmetic; bf16 or fp32 features.
+#include "bsa_internal.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int KN = 16;      // neighbours per target (4 x 4)
+constexpr double kPiD = 3.14159265358979323846;
+
+__global__ void __launch_bounds__(256)
+healpix_plan_kernel(int64_t nside, int64_t nlat, int64_t nlon, int32_t *__restrict__ nbr, float *__restrict__ rel) {
+    const int64_t npix = 12 * nside * nside;
+    const int64_t p = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (p >= npix) return;
+    const int face_row[12] = {2, 2, 2, 2, 3, 3, 3, 3, 4, 4, 4, 4};
+    const int face_col[12] = {1, 3, 5, 7, 0, 2, 4, 6, 1, 3, 5, 7};
+    const int64_t per_face = nside * nside;
+    const int f = (int)(p / per_face);
+    const int64_t ipf = p - f * per_face;
+    int64_t x = 0, y = 0;
+    for (int b = 0; ((int64_t)1 << (2 * b)) < per_face; ++b) {
+        x |= ((ipf >> (2 * b)) & 1) << b;
+        y |= ((ipf >> (2 * b + 1)) & 1) << b;
+    }
+    const int64_t ring = face_row[f] * nside - x - y - 1;
+    int64_t nr;
+    double z;
+    if (ring < nside) {
+        nr = ring;
+        z = 1.0 - (double)(nr * nr) / (3.0 * (double)per_face);
+    } else if (ring > 3 * nside) {
+        nr = 4 * nside - ring;
+        z = -1.0 + (double)(nr * nr) / (3.0 * (double)per_face);
+    } else {
+        nr = nside;
+        z = 4.0 / 3.0 - 2.0 * (double)ring / (3.0 * (double)nside);
+    }
+    double phi = (double)(face_col[f] * nr + (x - y)) * (kPiD / 4.0) / (double)nr;
+    if (phi < 0.0) phi += 2.0 * kPiD;
+    if (phi >= 2.0 * kPiD) phi -= 2.0 * kPiD;
+    const double dlat = 180.0 / (double)(nlat - 1), dlon = 360.0 / (double)nlon;
+    const double h = dlat * kPiD / 180.0;
+    const double lat = asin(z) * 180.0 / kPiD, lon = phi * 180.0 / kPiD;
+    const double st = sqrt(1.0 - z * z);
+    const double xi0 = st * cos(phi), xi1 = st * sin(phi), xi2 = z;
+    int64_t r0 = (int64_t)floor((90.0 - lat) / dlat) - 1;
+    r0 = r0 < 0 ? 0 : (r0 > nlat - 4 ? nlat - 4 : r0);
+    const int64_t c0 = (int64_t)floor(lon / dlon);
+    for (int a = 0; a < 4; ++a) {
+        const int64_t r = r0 + a;
+        const double la = (90.0 - (double)r * dlat) * kPiD / 180.0;
+        const double cl = cos(la), sl = sin(la);
+        for (int b = 0; b < 4; ++b) {
+            const int64_t c = ((c0 - 1 + b) % nlon + nlon) % nlon;
+            const int64_t e = p * KN + a * 4 + b;
+            nbr[e] = (int32_t)(r * nlon + c);
+            const double lo = (double)c * dlon * kPiD / 180.0;
+            rel[e * 3] = (float)((cl * cos(lo) - xi0) / h);
+            rel[e * 3 + 1] = (float)((cl * sin(lo) - xi1) / h);
+            rel[e * 3 + 2] = (float)((sl - xi2) / h);
+        }
+    }
+}
+
+template <typename T> __device__ __forceinline__ float load1(const T *p);
+template <> __device__ __forceinline__ float load1<float>(const float *p) { return __ldg(p); }
+template <> __device__ __forceinline__ float load1<__nv_bfloat16>(const __nv_bfloat16 *p) {
+    return __bfloat162float(*p);
+}
+
+template <typename T, int C>
+__global__ void __launch_bounds__(256)
+interp_kernel(int64_t n_tgt, int64_t n_src, const int32_t *__restrict__ nbr, const float *__restrict__ rel,
+              const float *__restrict__ wq, const T *__restrict__ ksrc, const T *__restrict__ vsrc,
+              T *__restrict__ out, float scale_log2, uint32_t *status) {
+    constexpr int D = 32 * C;
+    const int lane = threadIdx.x & 31;
+    const int64_t batch = blockIdx.y;
+    const T *kb = ksrc + batch * n_src * D, *vb = vsrc + batch * n_src * D;
+    float w[C][3];
+#pragma unroll
+    for (int c = 0; c < C; ++c)
+#pragma unroll
+        for (int e = 0; e < 3; ++e) w[c][e] = __ldg(wq + (lane * C + c) * 3 + e);
+    for (int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; i < n_tgt;
+         i += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+        int32_t src[KN];
+        float lg[KN];
+        bool bad = false;
+#pragma unroll
+        for (int j = 0; j < KN; ++j) {
+            src[j] = __ldg(nbr + i * KN + j);
+            if (src[j] < 0 || src[j] >= n_src) {
+                bad = true;
+                src[j] = 0;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < KN; ++j) {
+            const float *pr = rel + (i * KN + j) * 3;
+            const float p0 = __ldg(pr), p1 = __ldg(pr + 1), p2 = __ldg(pr + 2);
+            const T *kr = kb + (int64_t)src[j] * D + lane * C;
+            float part = 0.f;
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                const float qc = fmaf(w[c][0], p0, fmaf(w[c][1], p1, w[c][2] * p2));
+                part = fmaf(qc, load1<T>(kr + c), part);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+            lg[j] = part * scale_log2;      // log2 domain
+        }
+        float mx = lg[0];
+#pragma unroll
+        for (int j = 1; j < KN; ++j) mx = fmaxf(mx, lg[j]);
+        float den = 0.f;
+#pragma unroll
+        for (int j = 0; j < KN; ++j) {
+            lg[j] = exp2f(lg[j] - mx);
+            den += lg[j];
+        }
+        const float inv = 1.f / den;
+        float acc[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) acc[c] = 0.f;
+#pragma unroll
+        for (int j = 0; j < KN; ++j) {
+            const T *vr = vb + (int64_t)src[j] * D + lane * C;
+#pragma unroll
+            for (int c = 0; c < C; ++c) acc[c] = fmaf(lg[j], load1<T>(vr + c), acc[c]);
+        }
+        T *o = out + (batch * n_tgt + i) * D + lane * C;
+#pragma unroll
+        for (int c = 0; c < C; ++c) o[c] = from_f32<T>(acc[c] * inv);
+        if (bad && lane == 0 && status) atomicOr(status, kStatusBadIndex);
+    }
+}
+
+template <typename T>
+cudaError_t launch_interp_t(int64_t batch, int64_t n_tgt, int64_t n_src, int64_t d, const int32_t *nbr,
+                            const float *rel, const float *wq, const void *k, const void *v, void *out, float scale,
+                            uint32_t *status, cudaStream_t stream) {
+    int64_t ctas = (n_tgt * 32 + 255) / 256;
+    if (ctas > 148 * 64) ctas = 148 * 64;
+    if (ctas < 1) ctas = 1;
+    const dim3 grid((unsigned)ctas, (unsigned)batch);
+    const float sl2 = scale * 1.4426950408889634f;
+    const T *kt = static_cast<const T *>(k), *vt = static_cast<const T *>(v);
+    T *ot = static_cast<T *>(out);
+    switch (d) {
+        case 32: interp_kernel<T, 1><<<grid, 256, 0, stream>>>(n_tgt, n_src, nbr, rel, wq, kt, vt, ot, sl2, status); break;
+        case 64: interp_kernel<T, 2><<<grid, 256, 0, stream>>>(n_tgt, n_src, nbr, rel, wq, kt, vt, ot, sl2, status); break;
+        case 128: interp_kernel<T, 4><<<grid, 256, 0, stream>>>(n_tgt, n_src, nbr, rel, wq, kt, vt, ot, sl2, status); break;
+        default: return cudaErrorNotSupported;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_healpix_plan(int64_t nside, int64_t nlat, int64_t nlon, int32_t *nbr, float *rel,
+                                cudaStream_t stream) {
+    const int64_t npix = 12 * nside * nside;
+    healpix_plan_kernel<<<(unsigned)((npix + 255) / 256), 256, 0, stream>>>(nside, nlat, nlon, nbr, rel);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_interp(int64_t batch, int64_t n_tgt, int64_t n_src, int64_t d, bsa_dtype dtype,
+                          const int32_t *nbr, const float *rel, const float *wq, const void *k, const void *v,
+                          void *out, float scale, uint32_t *status, cudaStream_t stream) {
+    if (dtype == BSA_BF16)
+        return launch_interp_t<__nv_bfloat16>(batch, n_tgt, n_src, d, nbr, rel, wq, k, v, out, scale, status, stream);
+    return launch_interp_t<float>(batch, n_tgt, n_src, d, nbr, rel, wq, k, v, out, scale, status, stream);
+}
+
+}  // namespace bsa

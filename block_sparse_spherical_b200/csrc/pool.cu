@@ -105,6 +105,10 @@ cudaError_t launch_pool(const Problem &p, const void *q, const void *k, const vo
                         float *qbar, float *kbar, float *vbar, cudaStream_t stream) {
     if (p.dtype == BSA_BF16 && p.block_size == 64 && p.head_dim == 64)
         return launch<__nv_bfloat16, 64, 64>(p, q, k, v, qbar, kbar, vbar, stream);
+    if (p.dtype == BSA_BF16 && p.block_size == 256 && p.head_dim == 64)
+        return launch<__nv_bfloat16, 256, 64>(p, q, k, v, qbar, kbar, vbar, stream);
+    if (p.dtype == BSA_BF16 && p.block_size == 1024 && p.head_dim == 64)
+        return launch<__nv_bfloat16, 1024, 64>(p, q, k, v, qbar, kbar, vbar, stream);
     if (p.dtype == BSA_F32 && p.block_size == 64 && p.head_dim == 64)
         return launch<float, 64, 64>(p, q, k, v, qbar, kbar, vbar, stream);
     if (p.dtype == BSA_F32 && p.block_size == 16 && p.head_dim == 32)

@@ -35,8 +35,8 @@
  *    with 1 <= top_n <= min(m, 64) and window_blocks >= 0. bf16 inputs use
  *    bf16 tensor-core products with fp32 accumulation; the compressed
  *    branch and the top-n decision are fp32-accurate (fp32 on the CUDA
- *    cores, or, for head_dim 64 and top_n 16, three-pass tf32 products on
- *    the tensor cores).
+ *    cores, or, for head_dim 64 and top_n 16 or 32, three-pass tf32 products
+ *    on the tensor cores).
  */
 #ifndef BSA_H
 #define BSA_H
@@ -94,7 +94,7 @@ BSA_API bsa_status bsa_pool(const bsa_config *cfg, const void *q, const void *k,
  *   z_ij = s·q̄_i·k̄_j,  o_cg_block[i] = Σ_j softmax_j(z_ij) v̄_j,
  *   sel_idx[i] = the top_n blocks j by (z_ij descending, j ascending).
  * The m×m logit matrix is never written to memory. For head_dim 64 and
- * top_n 16 the products run on the tensor cores as three tf32 products each
+ * top_n 16 or 32 the products run on the tensor cores as three tf32 products each
  * (operands split into tf32 high and low parts); other shapes use fp32 on the
  * CUDA cores. The tensor-core kernel bounds every internal wait (2 s); should
  * one expire, the affected rows get -1 as their block indices (which
@@ -154,6 +154,117 @@ BSA_API bsa_status bsa_forward(const bsa_config *cfg, const void *q, const void 
  * or BSA_ERR_INDEX (BSA_ERR_CUDA if the copy itself fails).
  */
 BSA_API bsa_status bsa_check_status(const void *status_word, cudaStream_t stream);
+
+/*
+ * bsa_forward whose fine-attention epilogue also stores every output row, at
+ * the same offset as in `out`, into n_mirrors further buffers (0..7; a host
+ * array of device pointers, 16-byte aligned, none equal to out): the
+ * all-gather of a forward sharded by (batch, head) slab over the GPUs of one
+ * node, done by the kernel's own stores as each tile finishes. In that use
+ * every rank passes, as `out` and mirrors, its slab range within its own and
+ * its peers' full output buffers (peer memory mapped over NVLink, e.g.
+ * symmetric memory); the caller synchronises the ranks afterwards (a system
+ * barrier) before reading peers' rows. bf16 only (the tensor-core kernel);
+ * otherwise as bsa_forward. Not a step of the method: its distribution.
+ */
+BSA_API bsa_status bsa_forward_mirrored(const bsa_config *cfg, const void *q, const void *k, const void *v,
+                                        const float *gates, void *out, void *const *mirrors, int32_t n_mirrors,
+                                        int32_t *sel_idx_out, void *workspace, size_t workspace_bytes,
+                                        cudaStream_t stream);
+
+/*
+ * Lat-lon -> HEALPix cross-attention interpolation, the step before BSA in
+ * the MOSAIC note's pipeline ("overall framework", step (1), and the HEALPix
+ * paragraph): every HEALPix target pixel i attends to its neighbouring source
+ * points j of a latitude-longitude grid, with the relative position p_ij as
+ * the query and the source features as keys and values,
+ *   o_i = Σ_{j in N_i} softmax_j((W_q p_ij)·k_j · s) v_j.
+ *
+ * bsa_latlon_healpix_plan: for the 12·nside² NESTED pixels (nside a power of
+ * two) over a grid of nlat rows (+90 .. -90 degrees, poles included) and nlon
+ * columns (0 degrees eastwards, source index row*nlon + col): N_i, the 4 x 4
+ * grid points around the pixel centre (rows r0..r0+3 with r0 = floor((90 -
+ * lat)/dlat) - 1 clamped to [0, nlat-4]; columns c0-1..c0+2 wrapping in
+ * longitude, c0 = floor(lon/dlon)), written to nbr [npix][16] int32, and
+ * p_ij = (x_j - x_i)/dlat_rad (unit vectors, grid step in radians) to rel
+ * [npix][16][3] float. Device buffers, 16-byte aligned.
+ *
+ * bsa_latlon_to_healpix: the attention over such a plan for `batch`
+ * independent feature sets: k_src, v_src [batch][n_src][head_dim] and out
+ * [batch][n_tgt][head_dim] in `dtype` (bf16 or fp32), wq [head_dim][3]
+ * float (the query map), scale 0 = 1/sqrt(head_dim); head_dim 32, 64 or 128.
+ * fp32 arithmetic. Neighbour indices outside [0, n_src) are replaced by 0 and
+ * flagged BSA_ERR_INDEX in *status_word (nullable).
+ */
+BSA_API bsa_status bsa_latlon_healpix_plan(int64_t nside, int64_t nlat, int64_t nlon, int32_t *nbr, float *rel,
+                                           cudaStream_t stream);
+BSA_API bsa_status bsa_latlon_to_healpix(int64_t batch, int64_t n_tgt, int64_t n_src, int64_t head_dim,
+                                         int32_t dtype, float scale, const int32_t *nbr, const float *rel,
+                                         const float *wq, const void *k_src, const void *v_src, void *out,
+                                         uint32_t *status_word, cudaStream_t stream);
+
+/*
+ * Token layouts other than HEALPix NESTED. The note's ablation "BSA but not
+ * HEALPix (lat-lon block)" takes the blocks from a latitude-longitude grid;
+ * BSA itself needs each block contiguous, so such a layout is brought into
+ * block-contiguous order before the forward and back after it:
+ *   dst[s][t][:] = src[s][perm[t]][:]   for every slab s < slabs, t < n_tokens
+ * Rows are row_bytes long (head_dim x element size, or 3 x 4 for gates; a
+ * multiple of 4), src and dst distinct device buffers of slabs*n_tokens rows
+ * (16-byte aligned when row_bytes is a multiple of 16, else 4-byte aligned),
+ * perm a device int32 [n_tokens] shared by all slabs (a
+ * permutation: entries outside [0, n_tokens) are skipped and flagged
+ * BSA_ERR_INDEX in *status_word, nullable). The inverse move uses the
+ * inverse permutation.
+ */
+BSA_API bsa_status bsa_permute_tokens(int64_t slabs, int64_t n_tokens, int64_t row_bytes, const int32_t *perm,
+                                      const void *src, void *dst, uint32_t *status_word, cudaStream_t stream);
+
+/*
+ * Training. The MOSAIC note trains its model through BSA ("loss function /
+ * training strategy" sections: autoregressive training on ERA5), so the
+ * library provides the gradient of the forward above. The top-n choice is a
+ * discrete decision and carries no gradient: the backward holds the selected
+ * blocks fixed, and the compressed branch carries the gradient to the pooled
+ * keys and values it attends over. bf16 with block_size 64 and head_dim 64
+ * only (BSA_ERR_UNSUPPORTED otherwise).
+ *
+ * bsa_forward_train: bsa_forward plus the tensors bsa_backward needs, all
+ * caller-owned device buffers (16-byte aligned):
+ *   sel_idx    [B][H][m][top_n] int32   selected blocks (as bsa_forward's sel_idx_out)
+ *   o_cg_block [B][H][m][d]     float   compressed-branch output per query block
+ *   lse_cg     [B][H][m]        float   ln Σ_j exp(z_ij) of each compressed row
+ *   o_fg, o_l  [B][H][N][d]     dtype   selection and local branch outputs (before the gates)
+ *   lse_fine   [B][H][N][2]     float   ln Σ_u exp(s·q_t·k_u) of each token over its
+ *                                       selected (index 0) and local (index 1) keys
+ * workspace as for bsa_forward (bsa_workspace_size bytes, status word first).
+ */
+BSA_API bsa_status bsa_forward_train(const bsa_config *cfg, const void *q, const void *k, const void *v,
+                                     const float *gates, void *out, int32_t *sel_idx, float *o_cg_block,
+                                     float *lse_cg, void *o_fg, void *o_l, float *lse_fine, void *workspace,
+                                     size_t workspace_bytes, cudaStream_t stream);
+
+/* Bytes of device workspace bsa_backward needs for cfg. */
+BSA_API bsa_status bsa_backward_workspace_size(const bsa_config *cfg, size_t *bytes);
+
+/*
+ * Gradients of L with respect to q, k, v and the gates, given dout = dL/dout
+ * ([B][H][N][d], dtype) and the tensors bsa_forward_train saved:
+ *   dq, dk, dv [B][H][N][d] dtype,  dgates [B][H][N][3] float (CG, FG, L).
+ * Chain rule through the combine (dgates_t = dout_t·(o_CG, o_FG, o_L)), the
+ * selection and local softmax rows, the compressed branch (block level) and
+ * the mean pooling (each token gets 1/block_size of its block's pooled
+ * gradient). Runs on `stream` with `workspace` (device, >= bsa_backward_workspace_size
+ * bytes, 256-byte aligned; its first 4 bytes are a status word, as in
+ * bsa_forward, read by bsa_check_status). Accumulates in fp32; dq, dk, dv
+ * are rounded to dtype once at the end. Block indices outside [0, m) in
+ * sel_idx are skipped and flagged BSA_ERR_INDEX in the status word.
+ */
+BSA_API bsa_status bsa_backward(const bsa_config *cfg, const void *q, const void *k, const void *v,
+                                const float *gates, const void *dout, const int32_t *sel_idx,
+                                const float *o_cg_block, const float *lse_cg, const void *o_fg, const void *o_l,
+                                const float *lse_fine, void *dq, void *dk, void *dv, float *dgates,
+                                void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Allocation-free variant of bsa_forward (the MOSAIC note has no counterpart:

@@ -27,6 +27,14 @@ BSA_API bsa_status bsa_testing_fine_attention_withhold(const bsa_config *cfg, co
                                                        void *out, uint32_t *status_word,
                                                        int64_t withhold_v_step, cudaStream_t stream);
 
+/*
+ * y[i] = 2^x[i] (n device floats) as the fine-attention kernel's softmax forms
+ * it: poly != 0 takes the FMA-pipe route (range reduction and a degree-3
+ * minimax polynomial), poly == 0 the exp unit (ex2.approx). Lets a test hold
+ * the polynomial to its error bound against exact 2^x and the exp unit.
+ */
+BSA_API bsa_status bsa_testing_exp2(const float *x, float *y, int64_t n, int32_t poly, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -77,7 +77,7 @@ def test_workspace_size_layout(lib):
         idx = cfg.slabs * cfg.n_blocks * cfg.top_n * 4
         up = lambda x: (x + 255) // 256 * 256
         split = 0
-        if cfg.head_dim == 64 and cfg.top_n == 16:   # tensor-core compressed path: tf32 split images
+        if cfg.head_dim == 64 and cfg.top_n in (16, 32):   # tensor-core compressed path: tf32 split images
             m = cfg.n_blocks
             row_tiles, key_tiles = (m + 127) // 128, (m + 63) // 64
             split = cfg.slabs * (row_tiles * 65536 + 2 * key_tiles * 32768)

@@ -73,6 +73,9 @@ EDGE = {
     "topn_equals_m": (64, 64, "bf16", 2048, 1, 2, 32, 1),
     "tc_compress_n_eq_m16": (64, 64, "bf16", 1024, 1, 2, 16, 1),
     "tc_compress_m257_ragged": (64, 64, "bf16", 64 * 257, 1, 3, 16, 2),
+    "bf16_block256_nside32": (256, 64, "bf16", 12288, 1, 2, 4, 1),
+    "bf16_block256_ragged_w2": (256, 64, "bf16", 256 * 37, 2, 1, 5, 2),
+    "bf16_block1024_m12": (1024, 64, "bf16", 1024 * 12, 1, 2, 3, 1),
     "f32_block64": (64, 64, "f32", 4096, 1, 2, 8, 1),
     "f32_tiny_n_eq_m": (16, 32, "f32", 768, 1, 2, 48, 1),
     "f32_tiny_ragged": (16, 32, "f32", 16 * 75, 3, 1, 5, 3),
@@ -212,3 +215,23 @@ def test_compress_with_workspace_matches(name):
     torch.cuda.synchronize()
     assert torch.equal(i1, i2)
     assert torch.equal(o1, o2)
+
+
+def test_mirrored_output_stores():
+    """bsa_forward_mirrored (the epilogue that also stores every output row into further
+    buffers, the fused all-gather of the sharded forward) writes bsa_forward's output, bit for
+    bit, into out and into each mirror; here the mirrors are local buffers."""
+    cfg = CONFIGS["nside32"]
+    q, k, v, g = parity.device_inputs(cfg)
+    ref = api.BSA.from_config(cfg)
+    want = ref(q, k, v, g)
+    c = abi.make_config(cfg)
+    nbytes = abi.bsa_workspace_size(c)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    out = torch.full_like(q, float("nan"))
+    mirrors = [torch.full_like(q, float("nan")) for _ in range(3)]
+    abi.bsa_forward_mirrored(c, q, k, v, g, out, mirrors, None, ws, nbytes)
+    torch.cuda.synchronize()
+    assert abi.bsa_check_status(ws) == 0
+    for t in [out] + mirrors:
+        assert torch.equal(t, want)
