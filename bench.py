@@ -512,6 +512,104 @@ def run_sharded(args, cfg, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def _event_ms(fn, steps, warmup, dev):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize(dev)
+    return a.elapsed_time(b) / steps
+
+
+def run_interp(args, rank, local_rank):
+    """Lat-lon -> HEALPix cross-attention interpolation: a 0.25 degree grid (721 x 1440) onto the
+    786,432 pixels of Nside 256, d = 64, bf16 features, batch 8 (the Nside 256 workload's heads).
+    One step = bsa_latlon_to_healpix over the plan (built once, outside the timed region)."""
+    import torch
+    from block_sparse_spherical_b200 import abi, api
+    if rank != 0:
+        return
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    nside, nlat, nlon, d, batch = 256, 721, 1440, 64, 8
+    g = torch.Generator(device=dev).manual_seed(9)
+    k = torch.randn((batch, nlat * nlon, d), generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn((batch, nlat * nlon, d), generator=g, device=dev).to(torch.bfloat16)
+    wq = (torch.randn((d, 3), generator=g, device=dev) / 3 ** 0.5).float()
+    layer = api.LatLonToHealpix(nside, nlat, nlon, device=dev)
+    out = torch.empty((batch, layer.npix, d), dtype=torch.bfloat16, device=dev)
+    plan_ms = _event_ms(lambda: abi.bsa_latlon_healpix_plan(nside, nlat, nlon, layer.nbr, layer.rel), 3, 1, dev)
+    ms = _event_ms(lambda: layer(k, v, wq, out=out), args.steps, args.warmup, dev)
+    npix = layer.npix
+    # bytes the kernel must move at least: the plan (16 indices + 48 floats per pixel), the output,
+    # and the gathered rows (16 neighbours' k and v per pixel), which come from L2 (source 2 x 133 MB)
+    plan_b = npix * (16 * 4 + 48 * 4)
+    out_b = batch * npix * d * 2
+    gather_b = batch * npix * 16 * 2 * d * 2
+    peaks, src = load_peaks()
+    line = {"metric": "lat-lon -> HEALPix interpolation pixels/s (0.25 deg grid onto Nside 256, d 64, bf16)",
+            "pass": "interp", "value": batch * npix / (ms / 1e3), "unit": "pixels/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "interp_0.25deg_to_nside256", "nlat": nlat, "nlon": nlon, "nside": nside,
+                       "head_dim": d, "batch": batch, "neighbours": 16},
+            "plan_ms": plan_ms,
+            "roofline": {"kernel": "interp_kernel", "bound": "hbm", "achieved": (plan_b + out_b) / (ms / 1e3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": (plan_b + out_b) / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                         "l2_gather_gbs": gather_b / (ms / 1e3) / 1e9, "peak_source": f"{src} hbm_gbs",
+                         "traffic": None},
+            "gpu_launches": args.steps, "gpu": torch.cuda.get_device_name(dev)}
+    print(json.dumps(line), flush=True)
+
+
+def run_latlon(args, cfg, rank, local_rank):
+    """BSA over lat-lon blocks (the note's "BSA but not HEALPix" ablation) at the workload's size:
+    N points of a 384 x 512 (Nside 128: 196,608) lat-lon grid in 8 x 8 patches. One step = permute q,
+    k, v, gates to block-contiguous order, bsa_forward, permute the output back."""
+    import torch
+    from block_sparse_spherical_b200 import abi, api, layouts
+    from block_sparse_spherical_b200.synthetic import make_inputs
+    if rank != 0:
+        return
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    grids = {12288: (96, 128), 49152: (192, 256), 196608: (384, 512), 786432: (768, 1024)}
+    nlat, nlon = grids[cfg.n_tokens]
+    perm = torch.from_numpy(layouts.latlon_patches(nlat, nlon, 8, 8)).to(dev)
+    inv = torch.from_numpy(layouts.inverse(layouts.latlon_patches(nlat, nlon, 8, 8))).to(dev)
+    host = lambda a: torch.from_numpy(a).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+    q, k, v, g = (host(a).to(dev) for a in make_inputs(cfg))
+    qp, kp, vp, gp = (torch.empty_like(x) for x in (q, k, v, g))
+    bsa = api.BSA.from_config(cfg, device=dev)
+    out, outr = torch.empty_like(q), torch.empty_like(q)
+    S, n = cfg.slabs, cfg.n_tokens
+
+    def step():
+        for src, dst in ((q, qp), (k, kp), (v, vp), (g, gp)):
+            abi.bsa_permute_tokens(S, n, src.shape[-1] * src.element_size(), perm, src, dst)
+        bsa(qp, kp, vp, gp, out=out)
+        abi.bsa_permute_tokens(S, n, out.shape[-1] * out.element_size(), inv, out, outr)
+
+    ms = _event_ms(step, args.steps, args.warmup, dev)
+    perm_b = 2 * (3 * q.numel() * q.element_size() + g.numel() * 4 + out.numel() * out.element_size())
+    fwd_ms = _event_ms(lambda: bsa(q, k, v, g, out=out), args.steps, args.warmup, dev)
+    line = {"metric": "BSA fwd tokens/s over lat-lon 8x8-patch blocks (permute, forward, permute back)",
+            "pass": "latlon", "value": cfg.batch * n / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": cfg.dtype, "data": "synthetic",
+            "config": dict(workload_config(cfg), grid=f"{nlat} x {nlon} lat-lon, 8 x 8 patches"),
+            "forward_alone_ms": fwd_ms, "permute_ms": ms - fwd_ms,
+            "permute_gbs": perm_b / ((ms - fwd_ms) / 1e3) / 1e9 if ms > fwd_ms else None,
+            "gpu_launches": 6 * args.steps, "gpu": torch.cuda.get_device_name(dev)}
+    print(json.dumps(line), flush=True)
+
+
 def run_backward(args, cfg, rank, world, local_rank):
     """Training pass: one step = bsa_backward (every backward kernel) on the saved tensors of one
     bsa_forward_train of the workload, with a seeded dout; the forward itself is not timed."""
@@ -590,8 +688,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
-                    help="backward: time the training gradient (bsa_backward) instead of the forward")
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward", "interp", "latlon"],
+                    help="backward: the training gradient (bsa_backward); interp: the lat-lon -> HEALPix "
+                         "interpolation; latlon: BSA over lat-lon patch blocks (with the permutations)")
     ap.add_argument("--shard", action="store_true",
                     help="split one problem's (batch, head) slabs over the ranks (strong scaling) instead of "
                          "running an independent replica per rank")
@@ -609,6 +708,10 @@ def main():
         run_reference(args, cfg, rank)
     elif args.which == "backward":
         run_backward(args, cfg, rank, world, local_rank)
+    elif args.which == "interp":
+        run_interp(args, rank, local_rank)
+    elif args.which == "latlon":
+        run_latlon(args, cfg, rank, local_rank)
     elif args.shard:
         run_sharded(args, cfg, rank, world, local_rank)
     else:

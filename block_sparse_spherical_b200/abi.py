@@ -22,7 +22,7 @@ STATUS_NAMES = {
 EXPORTS = ("bsa_pool", "bsa_compress_select", "bsa_compress_select_ws", "bsa_fine_attention",
            "bsa_workspace_size", "bsa_forward", "bsa_check_status", "bsa_status_string", "bsa_forward_noalloc",
            "bsa_forward_train", "bsa_backward_workspace_size", "bsa_backward", "bsa_permute_tokens",
-           "bsa_latlon_healpix_plan", "bsa_latlon_to_healpix", "bsa_forward_mirrored")
+           "bsa_latlon_healpix_plan", "bsa_latlon_workspace_size", "bsa_latlon_to_healpix", "bsa_forward_mirrored")
 TESTING_EXPORTS = ("bsa_testing_fine_attention_withhold", "bsa_testing_exp2")
 
 
@@ -66,8 +66,9 @@ def load() -> ctypes.CDLL:
         "bsa_permute_tokens": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P, P, P, P],
         "bsa_latlon_healpix_plan": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P, P],
         "bsa_forward_mirrored": [C, P, P, P, P, P, ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, P, P, S, P],
+        "bsa_latlon_workspace_size": [ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)],
         "bsa_latlon_to_healpix": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
-                                  ctypes.c_float, P, P, P, P, P, P, P, P],
+                                  ctypes.c_float, P, P, P, P, P, P, P, S, P, P],
         "bsa_testing_fine_attention_withhold": [C, P, P, P, P, P, P, P, P, ctypes.c_int64, P],
         "bsa_testing_exp2": [P, P, ctypes.c_int64, ctypes.c_int32, P],
     }
@@ -183,11 +184,18 @@ def bsa_latlon_healpix_plan(nside: int, nlat: int, nlon: int, nbr, rel, stream=N
                                                                      _stream(stream)))
 
 
+def bsa_latlon_workspace_size(batch: int, n_src: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check("bsa_latlon_workspace_size", load().bsa_latlon_workspace_size(batch, n_src, ctypes.byref(n)))
+    return n.value
+
+
 def bsa_latlon_to_healpix(batch: int, n_tgt: int, n_src: int, head_dim: int, dtype: int, scale: float, nbr, rel,
-                          wq, k_src, v_src, out, status_word=None, stream=None) -> None:
+                          wq, k_src, v_src, out, workspace, workspace_bytes: int, status_word=None,
+                          stream=None) -> None:
     _check("bsa_latlon_to_healpix", load().bsa_latlon_to_healpix(
         batch, n_tgt, n_src, head_dim, dtype, scale, _ptr(nbr), _ptr(rel), _ptr(wq), _ptr(k_src), _ptr(v_src),
-        _ptr(out), _ptr(status_word), _stream(stream)))
+        _ptr(out), _ptr(workspace), workspace_bytes, _ptr(status_word), _stream(stream)))
 
 
 def bsa_forward_mirrored(cfg: BsaConfig, q, k, v, gates, out, mirrors, sel_idx_out, workspace,

@@ -144,6 +144,7 @@ class LatLonToHealpix:
         self.nbr = torch.empty((self.npix, 16), dtype=torch.int32, device=device)
         self.rel = torch.empty((self.npix, 16, 3), dtype=torch.float32, device=device)
         abi.bsa_latlon_healpix_plan(nside, nlat, nlon, self.nbr, self.rel)
+        self._ws = None            # the keys' 3-float position-space images, sized on first use
 
     def __call__(self, k_src, v_src, wq, scale: float = 0.0, out=None, status_word=None):
         b, n_src, d = k_src.shape
@@ -155,8 +156,11 @@ class LatLonToHealpix:
         if out is None:
             out = torch.empty((b, self.npix, d), dtype=k_src.dtype, device=k_src.device)
         _require(out, "out", k_src.dtype, (b, self.npix, d))
+        need = abi.bsa_latlon_workspace_size(b, n_src)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=k_src.device)
         abi.bsa_latlon_to_healpix(b, self.npix, n_src, d, _dtype_code(k_src), scale, self.nbr, self.rel, wq, k_src,
-                                  v_src, out, status_word)
+                                  v_src, out, self._ws, self._ws.numel(), status_word)
         return out
 
 

@@ -1,39 +1,50 @@
-// Backward of softmax attention on the sm_100a tensor cores, organised by key
-// tile, for the two places BSA (MOSAIC note, BSA section) runs attention
-// between 64-row tiles: the selection and local branches (query block i
-// against key block j, token level) and the compressed branch (query tile I
-// of 64 pooled blocks against key tile J, block level, over all tiles).
+// Backward of softmax attention on the sm_100a tensor cores, for the two places
+// BSA (MOSAIC note, BSA section) runs attention between 64-row tiles: the
+// selection and local branches (query tiles against key tiles, token level) and
+// the compressed branch (tiles of 64 pooled blocks, all against all).
 //
-// For one key tile J and each query tile I that attends to it (a "step"),
-// with the forward's row log-sum-exp lse, the row term D = g·(dout·o) and the
-// branch gate g of every query row (g = 1 for the compressed branch, whose
-// incoming gradient dO_CG already carries g_CG):
+// For a query tile I and a key tile J that attends to it (a "step"), with the
+// forward's row log-sum-exp lse, the row term D = g·(dout·o) and the branch
+// gate g of every query row (g = 1 for the compressed branch, whose incoming
+// gradient dO_CG already carries g_CG):
 //   S  = Q_I K_Jᵀ,  dP = dO_I V_Jᵀ                 (tcgen05.mma, M=N=K=64)
 //   P  = exp(s·S - lse),  Pg = g·P,  dS = s·P∘(g·dP - D)      (CUDA cores)
-//   dV_J += Pgᵀ dO_I,  dK_J += dSᵀ Q_I              (accumulated in TMEM)
-//   dQ_I  = dS K_J                                  (TMEM, then added into an
-//                                                    fp32 dq accumulator with
-//                                                    vector reductions)
+//   dV_J += Pgᵀ dO_I,  dK_J += dSᵀ Q_I,  dQ_I += dS K_J
 // Pg and dS go to shared memory as bf16 rows (the MMA's K-major 128-byte
-// swizzle), which the two dV/dK MMAs read as transposed (MN-major) A operands
-// and the dQ MMA as a K-major one. dK_J and dV_J are complete when the key
-// tile's last step is; the epilogue writes them (token level: bf16, plus the
-// key block's share dk̄/B, dv̄/B of the pooled gradients; block level: fp32).
+// swizzle), which the dV/dK MMAs read as transposed (MN-major) A operands and
+// the dQ MMA as a K-major one.
 //
-// Key tiles are the units of work, handed out round-robin to two independent
-// pipelines per CTA (persistent grid, one CTA per SM). Per pipeline:
+// Three passes of one kernel:
+//   compressed (key-major, dense): units are key tiles J, steps every query tile
+//     (keys past m masked); dK_J, dV_J accumulate in TMEM and are written fp32 at
+//     the unit's end; dQ of each step is reduced into an fp32 dq̄ (small: one
+//     row per block) with red.global.add.v4.f32.
+//   fine key-major: units are key tiles J, steps the query tiles of J's block's
+//     clamped window, then of the query blocks whose top-n holds it (the
+//     selection inverted per slab); dK_J, dV_J accumulate in TMEM and are written
+//     bf16 with the block's 1/B share of dk̄, dv̄. No dQ here.
+//   fine query-major: units are query tiles I, steps the key tiles of its
+//     block's selected blocks, then of its window (the forward's order); dQ_I
+//     accumulates in TMEM and is written bf16 with the block's 1/B share of dq̄.
+//     Recomputing S and dP here costs two MMAs a step but keeps dq free of
+//     atomic reductions over the full token range.
+// No atomics on dk, dv or dq: all three are bit-for-bit deterministic.
+//
+// Units are handed out round-robin to two independent pipelines per CTA
+// (persistent grid, one CTA per SM). Per pipeline:
 //   warp p (0-1)        : MMA warp (one elected lane issues)
-//   warp 2+p            : TMA copy warp: K_J and V_J per unit (two buffers),
-//                         Q_I and dO_I per step (two stages)
+//   warp 2+p            : TMA copy warp: the unit's two tiles (key-major: K, V;
+//                         query-major: Q, dO; two buffers) and the step's two
+//                         (key-major: Q, dO; query-major: K, V; two stages)
 //   warps 4+4p..7+4p    : 128 softmax threads; thread (w, lane) owns row
 //                         16(w%4) + lane%16 and columns 32(lane/16)..+31 of
-//                         the step's S and dP, and the same rows/columns of
-//                         dQ, dK, dV
+//                         the step's S and dP, and of the unit's accumulators
 // Tensor memory (M=64 accumulators use 16 of the 32 lanes of each
 // sub-partition, so two share columns in the two lane halves):
 //   pipeline p: S  cols 128p..+63 lanes +0,  dP cols 128p..+63 lanes +16,
-//               dK cols 128p+64..+63 lanes +0, dV cols 128p+64..+63 lanes +16
-//   dQ of pipeline p: cols 256..319, lanes +16p
+//               dK (query-major: dQ) cols 128p+64..+63 lanes +0,
+//               dV cols 128p+64..+63 lanes +16
+//   per-step dQ of the compressed pass, pipeline p: cols 256..319, lanes +16p
 // Every wait on an mbarrier is bounded (2 s); on expiry the kernel records a
 // timeout in the status word, the other roles stop at their next wait, the
 // copies and MMAs in flight are drained, TMEM is freed and the kernel returns.
@@ -52,8 +63,18 @@ using namespace tc;
 constexpr int BK = 64;                     // rows of a tile
 constexpr int HD = 64;                     // head dim
 constexpr int TILE = BK * HD * 2;          // bytes of one 64x64 bf16 tile
-constexpr int NPIPE = 2;
+#ifndef BSA_BWD_PIPES
+#define BSA_BWD_PIPES 2
+#endif
+constexpr int NPIPE = BSA_BWD_PIPES;       // independent pipelines per CTA (2 or 3)
 constexpr int NTHREADS = 32 * (2 * NPIPE + 4 * NPIPE);
+// With three pipelines the unit tiles and the g·P / s·dS rows are single-buffered (64 KB of
+// shared memory a pipeline), and a register split gives the softmax threads their registers.
+constexpr int UB = NPIPE == 3 ? 1 : 2;     // unit tile buffers
+constexpr int DB = NPIPE == 3 ? 1 : 2;     // g·P / s·dS buffers
+constexpr int kCtrlRegs = 64, kSoftRegs = 112;
+constexpr int kRegsNeeded = 2 * NPIPE * 32 * kCtrlRegs + 4 * NPIPE * 32 * kSoftRegs;
+static_assert(NPIPE == 2 || kRegsNeeded <= 65536, "register split");
 constexpr uint32_t TMEM_COLS = 512;
 
 // instruction descriptors: D f32, A and B bf16, M = 64, N = 64
@@ -64,13 +85,13 @@ constexpr uint32_t kIdescTT = kIdesc | (1u << 15) | (1u << 16); // A, B MN-major
 constexpr uint32_t kIdescNT = kIdesc | (1u << 16);              // A K-major, B MN-major
 
 struct alignas(1024) PipeTiles {
-    uint8_t k[2][TILE], v[2][TILE];        // [unit buffer]
-    uint8_t q[2][TILE], o[2][TILE];        // [step stage]: Q_I and dO_I
-    uint8_t pg[2][TILE], ds[2][TILE];      // [step buffer]: g·P and s·dS rows
+    uint8_t u0[UB][TILE], u1[UB][TILE];    // [unit buffer]: K, V (key-major) or Q, dO (query-major)
+    uint8_t s0[2][TILE], s1[2][TILE];      // [step stage]: Q, dO (key-major) or K, V (query-major)
+    uint8_t pg[DB][TILE], ds[DB][TILE];    // [step buffer]: g·P and s·dS rows
 };
 struct PipeBars {
-    uint64_t kv_full[2], kv_empty[2];
-    uint64_t qo_full[2], qo_empty[2];
+    uint64_t ut_full[2], ut_empty[2];
+    uint64_t st_full[2], st_empty[2];
     uint64_t s_full, s_free;
     uint64_t ds_full[2], ds_empty[2];
     uint64_t dq_full, dq_free;
@@ -86,19 +107,23 @@ struct SharedStorage {
 
 struct BwdParams {
     int dense;               // 1: compressed branch (every query tile, one branch); 0: fine branches
+    int qmajor;              // 1: units are query tiles and the pass forms dQ only (fine branches)
+    int with_dq;             // key-major pass: also form dQ per step and reduce it into dq_acc
     int64_t rows;            // rows per slab of the operand tensors (dense: m_pad, fine: N)
-    int tiles;               // key tiles (= query tiles) per slab
+    int tiles;               // 64-row tiles per slab
     int64_t units;           // slabs * tiles
     int valid;               // rows per slab that exist (dense: m): later keys are masked
     int m, n, w;             // fine: blocks per slab, top-n, window (in blocks)
     int R;                   // fine: 64-row tiles per block (block_size / 64)
-    const int *offs, *list;  // fine: the inverted selection (per slab: m+1 offsets, m*n entries)
+    const int *offs, *list;  // key-major fine: the inverted selection (per slab: m+1 offsets, m*n entries)
+    const int32_t *idx;      // query-major: the selection [slabs*m][n]
     const float *lse;        // dense: [slabs*m_pad]; fine: [slabs*N][2] (FG, L)
     const float *dterm;      // D, same layout as lse
     const float *gates;      // fine: [slabs*N][3]; dense: null
-    float *dq_acc;           // [slabs*rows][64], reduced into
-    __nv_bfloat16 *dk, *dv;  // fine outputs [slabs*N][64]
-    const float *dkbar, *dvbar;   // fine: [slabs*m_pad][64], added as 1/B shares
+    float *dq_acc;           // key-major with_dq: [slabs*rows][64], reduced into
+    __nv_bfloat16 *dk, *dv;  // key-major fine outputs [slabs*N][64]
+    __nv_bfloat16 *dq;       // query-major output [slabs*N][64]
+    const float *dkbar, *dvbar, *dqbar;   // fine: [slabs*m_pad][64], added as 1/B shares
     int64_t m_pad;
     float inv_block;
     float *dk32, *dv32;      // dense outputs [slabs*m_pad][64]
@@ -106,56 +131,88 @@ struct BwdParams {
     uint32_t *status;        // nullable
 };
 
-// Step s of the unit with slab `slab` and key tile J: its query tile and branch
-// (0: selection / compressed, 1: local). Fine units run the tiles of the clamped
-// window's query blocks first, then the tiles of the query blocks that selected
-// J's block.
+// A unit: tile T of slab `slab` (the key tile of a key-major pass, the query tile of
+// a query-major one) and its steps. Key-major fine units run the query tiles of
+// T's block's clamped window, then those of the query blocks that selected it;
+// query-major units run the key tiles of the selected blocks, then of the window.
 struct Unit {
     int64_t slab;
-    int J, jb, lo, nloc, nsteps;   // key tile, its block, first window block, window steps
-    int64_t list_base;             // fine: first list entry of block jb
+    int T, tb, lo, nloc, nsteps;   // tile, its block, first window block, window steps (key-major)
+    int64_t list_base;             // key-major fine: first list entry of block tb
+    const int32_t *sel;            // query-major: the selected blocks of block tb
+};
+struct Step {
+    int tile;                      // the other side's tile
+    int branch;                    // 0: selection / compressed, 1: local
+    bool valid;                    // false: a selected block outside [0, m) (no keys)
 };
 __device__ __forceinline__ Unit unit_of(const BwdParams &p, int64_t u) {
     Unit x;
     x.slab = u / p.tiles;
-    x.J = (int)(u - x.slab * p.tiles);
+    x.T = (int)(u - x.slab * p.tiles);
+    x.lo = x.nloc = 0;
+    x.list_base = 0;
+    x.sel = nullptr;
     if (p.dense) {
-        x.nloc = 0;
+        x.tb = x.T;
         x.nsteps = p.tiles;
-        x.list_base = 0;
+    } else if (p.qmajor) {
+        x.tb = x.T / p.R;
+        x.sel = p.idx + (x.slab * p.m + x.tb) * (int64_t)p.n;
+        x.nsteps = (p.n + 2 * p.w + 1) * p.R;
     } else {
-        x.jb = x.J / p.R;
-        x.lo = max(0, x.jb - p.w);
-        const int hi = min(p.m - 1, x.jb + p.w);
+        x.tb = x.T / p.R;
+        x.lo = max(0, x.tb - p.w);
+        const int hi = min(p.m - 1, x.tb + p.w);
         x.nloc = (hi - x.lo + 1) * p.R;
         const int *o = p.offs + x.slab * (p.m + 1);
-        const int b = __ldg(o + x.jb);
+        const int b = __ldg(o + x.tb);
         x.list_base = x.slab * (int64_t)p.m * p.n + b;
-        x.nsteps = x.nloc + (__ldg(o + x.jb + 1) - b) * p.R;
+        x.nsteps = x.nloc + (__ldg(o + x.tb + 1) - b) * p.R;
     }
     return x;
 }
-__device__ __forceinline__ int step_tile(const BwdParams &p, const Unit &x, int s, int *branch) {
+__device__ __forceinline__ Step step_of(const BwdParams &p, const Unit &x, int s) {
+    Step st;
+    st.valid = true;
     if (p.dense) {
-        *branch = 0;
-        return s;
+        st.tile = s;
+        st.branch = 0;
+    } else if (p.qmajor) {
+        const int nr = p.n * p.R;
+        int j;
+        if (s < nr) {
+            j = __ldg(x.sel + s / p.R);
+            st.branch = 0;
+        } else {
+            j = x.tb - p.w + (s - nr) / p.R;
+            st.branch = 1;
+        }
+        st.valid = j >= 0 && j < p.m;
+        st.tile = st.valid ? j * p.R + s % p.R : x.T;   // an invalid block loads a harmless tile
+    } else if (s < x.nloc) {
+        st.tile = x.lo * p.R + s;
+        st.branch = 1;
+    } else {
+        const int e = s - x.nloc;
+        st.tile = __ldg(p.list + x.list_base + e / p.R) * p.R + e % p.R;
+        st.branch = 0;
     }
-    if (s < x.nloc) {
-        *branch = 1;
-        return x.lo * p.R + s;
-    }
-    *branch = 0;
-    const int e = s - x.nloc;
-    return __ldg(p.list + x.list_base + e / p.R) * p.R + e % p.R;
+    return st;
 }
 
 // ------------------------------------------------------------------ roles
 
+// Unit tiles (key-major: K_T, V_T; query-major: Q_T, dO_T) per unit, two buffers;
+// step tiles (key-major: Q, dO of the step's query tile; query-major: K, V of the
+// step's key tile) per step, two stages.
 __device__ void loader_role(const BwdParams &p, const CUtensorMap *tq, const CUtensorMap *tk, const CUtensorMap *tv,
                             const CUtensorMap *to, PipeTiles &S, PipeBars &B, int pipe, volatile int *abort_flag) {
     const int64_t stride = NPIPE * (int64_t)gridDim.x;
+    const CUtensorMap *u0 = p.qmajor ? tq : tk, *u1 = p.qmajor ? to : tv;
+    const CUtensorMap *s0 = p.qmajor ? tk : tq, *s1 = p.qmajor ? tv : to;
     uint32_t c = 0, g = 0;
-    uint64_t *last_bar[2] = {nullptr, nullptr};   // most recent K/V and Q/dO copies
+    uint64_t *last_bar[2] = {nullptr, nullptr};   // most recent unit and step copies
     uint32_t last_par[2] = {0, 0};
     bool ok = true;
     const bool leader = elect_one();
@@ -165,28 +222,30 @@ __device__ void loader_role(const BwdParams &p, const CUtensorMap *tq, const CUt
     for (int64_t u = NPIPE * (int64_t)blockIdx.x + pipe; u < p.units && ok; u += stride, ++c) {
         const Unit x = unit_of(p, u);
         const int64_t base = x.slab * p.rows;
-        const int kb = c & 1;
-        if (!(ok = wait_w(&B.kv_empty[kb], ((c >> 1) & 1) ^ 1))) break;
+        const int kb = c % UB;
+        if (!(ok = wait_w(&B.ut_empty[kb], ((c / UB) & 1) ^ 1))) break;
         if (leader) {
-            mbar_expect_tx(&B.kv_full[kb], 2 * TILE);
-            tma_load_tile(S.k[kb], tk, &B.kv_full[kb], (int)(base + (int64_t)x.J * BK));
-            tma_load_tile(S.v[kb], tv, &B.kv_full[kb], (int)(base + (int64_t)x.J * BK));
+            mbar_expect_tx(&B.ut_full[kb], 2 * TILE);
+            tma_load_tile(S.u0[kb], u0, &B.ut_full[kb], (int)(base + (int64_t)x.T * BK));
+            tma_load_tile(S.u1[kb], u1, &B.ut_full[kb], (int)(base + (int64_t)x.T * BK));
         }
         __syncwarp();
-        last_bar[0] = &B.kv_full[kb];
-        last_par[0] = (c >> 1) & 1;
+        last_bar[0] = &B.ut_full[kb];
+        last_par[0] = (c / UB) & 1;
         for (int s = 0; s < x.nsteps; ++s, ++g) {
-            int br;
-            const int I = step_tile(p, x, s, &br);
+            const Step stp = step_of(p, x, s);
             const int st = g & 1;
-            if (!(ok = wait_w(&B.qo_empty[st], ((g >> 1) & 1) ^ 1))) break;
+            // a selected block outside [0, m) is an error in the caller's indices; a window
+            // block past either end of the sequence is the clamping, not an error
+            if (leader && !stp.valid && stp.branch == 0 && p.status) atomicOr(p.status, kStatusBadIndex);
+            if (!(ok = wait_w(&B.st_empty[st], ((g >> 1) & 1) ^ 1))) break;
             if (leader) {
-                mbar_expect_tx(&B.qo_full[st], 2 * TILE);
-                tma_load_tile(S.q[st], tq, &B.qo_full[st], (int)(base + (int64_t)I * BK));
-                tma_load_tile(S.o[st], to, &B.qo_full[st], (int)(base + (int64_t)I * BK));
+                mbar_expect_tx(&B.st_full[st], 2 * TILE);
+                tma_load_tile(S.s0[st], s0, &B.st_full[st], (int)(base + (int64_t)stp.tile * BK));
+                tma_load_tile(S.s1[st], s1, &B.st_full[st], (int)(base + (int64_t)stp.tile * BK));
             }
             __syncwarp();
-            last_bar[1] = &B.qo_full[st];
+            last_bar[1] = &B.st_full[st];
             last_par[1] = (g >> 1) & 1;
         }
     }
@@ -201,53 +260,67 @@ __device__ void mma_role(const BwdParams &p, PipeTiles &S, PipeBars &B, uint32_t
     const int64_t stride = NPIPE * (int64_t)gridDim.x;
     const uint32_t tp = tmem + 128u * pipe;
     const uint32_t tS = tp, tdP = tp + (16u << 16), tdK = tp + 64, tdV = tp + 64 + (16u << 16);
-    const uint32_t tdQ = tmem + 256 + ((16u * pipe) << 16);
+    const uint32_t tdQ = tmem + 128u * NPIPE + 64u * (pipe >> 1) + ((16u * (pipe & 1)) << 16);
     uint32_t c = 0, g = 0;
     bool ok = true;
     const bool leader = elect_one();
     auto wait_w = [&](uint64_t *b, uint32_t par) -> bool {
         return __all_sync(0xffffffffu, wait_fast(b, par, abort_flag, p.status));
     };
-    // dV, dK and dQ of step gg (first: the unit's first step, which starts dK and dV afresh)
+    // the gradient MMAs of step gg (first: the unit's first step, which starts its
+    // accumulators afresh). Key-major: dV += Pgᵀ·dO, dK += dSᵀ·Q (+ dQ = dS·K per step);
+    // query-major: dQ += dS·K, accumulated in the dK columns.
     auto issue_grad = [&](uint32_t gg, bool first, int kb) -> bool {
-        const int b = gg & 1;
-        if (!wait_w(&B.ds_full[b], (gg >> 1) & 1)) return false;
+        const int b = gg % DB, st = gg & 1;
+        if (!wait_w(&B.ds_full[b], (gg / DB) & 1)) return false;
         if (first && c > 0 && !wait_w(&B.acc_free, (c - 1) & 1)) return false;
-        if (gg > 0 && !wait_w(&B.dq_free, (gg - 1) & 1)) return false;
+        if (p.with_dq && gg > 0 && !wait_w(&B.dq_free, (gg - 1) & 1)) return false;
         fence_after();
         if (leader) {
-            const uint64_t dpg = desc_mnmajor_sw128(S.pg[b], TILE), dds_t = desc_mnmajor_sw128(S.ds[b], TILE);
             const uint64_t dds = desc_kmajor_sw128(S.ds[b]);
-            const uint64_t dO = desc_mnmajor_sw128(S.o[b], TILE), dQm = desc_mnmajor_sw128(S.q[b], TILE);
-            const uint64_t dKm = desc_mnmajor_sw128(S.k[kb], TILE);
+            if (p.qmajor) {
+                const uint64_t dKm = desc_mnmajor_sw128(S.s0[st], TILE);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)        // K chunk kk: query rows 16kk..16kk+15
-                mma_bf16(tdV, dpg + 128 * kk, dO + 128 * kk, kIdescTT, (first && kk == 0) ? 0u : 1u);
+                for (int kk = 0; kk < 4; ++kk)    // K chunk kk: key columns 16kk..16kk+15
+                    mma_bf16(tdK, dds + 2 * kk, dKm + 128 * kk, kIdescNT, (first && kk == 0) ? 0u : 1u);
+            } else {
+                const uint64_t dpg = desc_mnmajor_sw128(S.pg[b], TILE), dds_t = desc_mnmajor_sw128(S.ds[b], TILE);
+                const uint64_t dO = desc_mnmajor_sw128(S.s1[st], TILE), dQm = desc_mnmajor_sw128(S.s0[st], TILE);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tdK, dds_t + 128 * kk, dQm + 128 * kk, kIdescTT, (first && kk == 0) ? 0u : 1u);
+                for (int kk = 0; kk < 4; ++kk)    // K chunk kk: query rows 16kk..16kk+15
+                    mma_bf16(tdV, dpg + 128 * kk, dO + 128 * kk, kIdescTT, (first && kk == 0) ? 0u : 1u);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)        // K chunk kk: key columns 16kk..16kk+15
-                mma_bf16(tdQ, dds + 2 * kk, dKm + 128 * kk, kIdescNT, kk > 0);
-            commit(&B.dq_full);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tdK, dds_t + 128 * kk, dQm + 128 * kk, kIdescTT, (first && kk == 0) ? 0u : 1u);
+                if (p.with_dq) {
+                    const uint64_t dKm = desc_mnmajor_sw128(S.u0[kb], TILE);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tdQ, dds + 2 * kk, dKm + 128 * kk, kIdescNT, kk > 0);
+                    commit(&B.dq_full);
+                }
+            }
             commit(&B.ds_empty[b]);
-            commit(&B.qo_empty[b]);
+            commit(&B.st_empty[st]);
         }
         __syncwarp();
         return true;
     };
     for (int64_t u = NPIPE * (int64_t)blockIdx.x + pipe; u < p.units && ok; u += stride, ++c) {
         const Unit x = unit_of(p, u);
-        const int kb = c & 1;
-        if (!(ok = wait_w(&B.kv_full[kb], (c >> 1) & 1))) break;
+        const int kb = c % UB;
+        if (!(ok = wait_w(&B.ut_full[kb], (c / UB) & 1))) break;
         for (int s = 0; s < x.nsteps; ++s, ++g) {
             const int st = g & 1;
-            if (!(ok = wait_w(&B.qo_full[st], (g >> 1) & 1))) break;
+            if (!(ok = wait_w(&B.st_full[st], (g >> 1) & 1))) break;
             if (g > 0 && !(ok = wait_w(&B.s_free, (g - 1) & 1))) break;
             fence_after();
             if (leader) {
-                const uint64_t dq = desc_kmajor_sw128(S.q[st]), dk = desc_kmajor_sw128(S.k[kb]);
-                const uint64_t dO = desc_kmajor_sw128(S.o[st]), dv = desc_kmajor_sw128(S.v[kb]);
+                // S = Q·Kᵀ and dP = dO·Vᵀ (Q, dO and K, V from the unit or the step tiles)
+                const uint8_t *q = p.qmajor ? S.u0[kb] : S.s0[st], *k = p.qmajor ? S.s0[st] : S.u0[kb];
+                const uint8_t *o = p.qmajor ? S.u1[kb] : S.s1[st], *v = p.qmajor ? S.s1[st] : S.u1[kb];
+                const uint64_t dq = desc_kmajor_sw128(q), dk = desc_kmajor_sw128(k);
+                const uint64_t dO = desc_kmajor_sw128(o), dv = desc_kmajor_sw128(v);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) mma_bf16(tS, dq + 2 * kk, dk + 2 * kk, kIdescNN, kk > 0);
 #pragma unroll
@@ -261,7 +334,7 @@ __device__ void mma_role(const BwdParams &p, PipeTiles &S, PipeBars &B, uint32_t
         if (x.nsteps > 0 && !(ok = issue_grad(g - 1, x.nsteps == 1, kb))) break;
         if (leader) {
             commit(&B.acc_full);
-            commit(&B.kv_empty[kb]);
+            commit(&B.ut_empty[kb]);
         }
         __syncwarp();
     }
@@ -276,6 +349,23 @@ __device__ __forceinline__ void red_add_v4(float *dst, float a, float b, float c
                  : "memory");
 }
 
+// 32 consecutive values as bf16 at dst: x[e] + f * add[e] (add nullable).
+__device__ __forceinline__ void store_row32_bf16(__nv_bfloat16 *dst, const float *x, const float *add, float f) {
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        uint32_t w[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const int cc = 8 * e + 2 * h;
+            const float a0 = add ? fmaf(__ldg(add + cc), f, x[cc]) : x[cc];
+            const float a1 = add ? fmaf(__ldg(add + cc + 1), f, x[cc + 1]) : x[cc + 1];
+            w[h] = pack_bf16x2(a0, a1);
+        }
+        d4[e] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 __device__ void softmax_role(const BwdParams &p, PipeTiles &S, PipeBars &B, uint32_t tmem, int pipe, int wq,
                              int lane, volatile int *abort_flag) {
     const unsigned FULL = 0xffffffffu;
@@ -286,7 +376,7 @@ __device__ void softmax_role(const BwdParams &p, PipeTiles &S, PipeBars &B, uint
     const uint32_t tp = tmem + 128u * pipe;
     const uint32_t tS = tp + (wl << 16), tdP = tp + ((wl + 16) << 16);
     const uint32_t tdK = tp + 64 + (wl << 16), tdV = tp + 64 + ((wl + 16) << 16);
-    const uint32_t tdQ = tmem + 256 + ((wl + 16u * pipe) << 16);
+    const uint32_t tdQ = tmem + 128u * NPIPE + 64u * (pipe >> 1) + ((wl + 16u * (pipe & 1)) << 16);
     const int prow_off = (r >> 3) * 1024 + (r & 7) * 128;
     const int sw = r & 7;
     const float sl2 = p.scale_log2, sc = p.scale;
@@ -314,8 +404,8 @@ __device__ void softmax_role(const BwdParams &p, PipeTiles &S, PipeBars &B, uint
         const Unit x = unit_of(p, u);
         int I_prev = 0;
         for (int s = 0; s < x.nsteps; ++s, ++g) {
-            int br;
-            const int I = step_tile(p, x, s, &br);
+            const Step stp = step_of(p, x, s);
+            const int I = p.qmajor ? x.T : stp.tile;   // the query tile of this step
             const int64_t row = x.slab * p.rows + (int64_t)I * BK + r;
             float lse2, D, gate;
             if (p.dense) {
@@ -323,9 +413,9 @@ __device__ void softmax_role(const BwdParams &p, PipeTiles &S, PipeBars &B, uint
                 D = __ldg(p.dterm + row);
                 gate = 1.f;
             } else {
-                lse2 = __ldg(p.lse + row * 2 + br) * 1.4426950408889634f;
-                D = __ldg(p.dterm + row * 2 + br);
-                gate = __ldg(p.gates + row * 3 + 1 + br);
+                lse2 = __ldg(p.lse + row * 2 + stp.branch) * 1.4426950408889634f;
+                D = __ldg(p.dterm + row * 2 + stp.branch);
+                gate = __ldg(p.gates + row * 3 + 1 + stp.branch);
             }
             // ---- S and dP of this step
             if (!(ok = wait_all(&B.s_full, g & 1))) break;
@@ -338,8 +428,9 @@ __device__ void softmax_role(const BwdParams &p, PipeTiles &S, PipeBars &B, uint
             tmem_wait_ld();
             fence_before();
             mbar_arrive(&B.s_free);
-            // keys past the slab's valid rows (block-level padding) take no part
-            const int kvalid = p.dense ? min(32, max(0, p.valid - (x.J * BK + 32 * ch))) : 32;
+            // keys that take no part: past the slab's valid rows (block-level padding), or
+            // of a selected block outside [0, m)
+            const int kvalid = p.dense ? min(32, max(0, p.valid - (x.T * BK + 32 * ch))) : (stp.valid ? 32 : 0);
             uint32_t ppk[16], dpk[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -351,66 +442,61 @@ __device__ void softmax_role(const BwdParams &p, PipeTiles &S, PipeBars &B, uint
                 ppk[e] = pack_bf16x2(gate * p0, gate * p1);
                 dpk[e] = pack_bf16x2(d0, d1);
             }
-            // ---- g·P and s·dS rows into buffer g%2 once the MMAs of step g-2 released it
-            const int b = g & 1;
-            if (!(ok = wait_all(&B.ds_empty[b], ((g >> 1) & 1) ^ 1))) break;
+            // ---- s·dS (and g·P) rows into buffer g%2 once the MMAs of step g-2 released it
+            const int b = g % DB;
+            if (!(ok = wait_all(&B.ds_empty[b], ((g / DB) & 1) ^ 1))) break;
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
                 const int chunk = 4 * ch + c4;
                 const int off = prow_off + ((chunk ^ sw) << 4);
-                *reinterpret_cast<uint4 *>(S.pg[b] + off) =
-                    make_uint4(ppk[4 * c4], ppk[4 * c4 + 1], ppk[4 * c4 + 2], ppk[4 * c4 + 3]);
+                if (!p.qmajor)
+                    *reinterpret_cast<uint4 *>(S.pg[b] + off) =
+                        make_uint4(ppk[4 * c4], ppk[4 * c4 + 1], ppk[4 * c4 + 2], ppk[4 * c4 + 3]);
                 *reinterpret_cast<uint4 *>(S.ds[b] + off) =
                     make_uint4(dpk[4 * c4], dpk[4 * c4 + 1], dpk[4 * c4 + 2], dpk[4 * c4 + 3]);
             }
             fence_proxy_async();
             fence_before();
             mbar_arrive(&B.ds_full[b]);
-            // ---- dQ of the previous step
-            if (s > 0 && !(ok = finish_dq(g - 1, x.slab, I_prev))) break;
+            // ---- dQ of the previous step (key-major pass with dQ)
+            if (p.with_dq && s > 0 && !(ok = finish_dq(g - 1, x.slab, I_prev))) break;
             I_prev = I;
         }
         if (!ok) break;
-        if (x.nsteps > 0 && !(ok = finish_dq(g - 1, x.slab, I_prev))) break;
-        // ---- epilogue: dK and dV of key tile J
+        if (p.with_dq && x.nsteps > 0 && !(ok = finish_dq(g - 1, x.slab, I_prev))) break;
+        // ---- epilogue of the unit
         if (!(ok = wait_all(&B.acc_full, c & 1))) break;
         fence_after();
         float dk[32], dv[32];
         tmem_ld16x2(tdK, dk);
         tmem_ld16x2(tdK + 16, dk + 16);
-        tmem_ld16x2(tdV, dv);
-        tmem_ld16x2(tdV + 16, dv + 16);
+        if (!p.qmajor) {
+            tmem_ld16x2(tdV, dv);
+            tmem_ld16x2(tdV + 16, dv + 16);
+        }
         tmem_wait_ld();
         fence_before();
         mbar_arrive(&B.acc_free);
-        const int64_t krow = x.slab * p.rows + (int64_t)x.J * BK + r;
-        if (p.dense) {
-            float4 *k4 = reinterpret_cast<float4 *>(p.dk32 + krow * HD + 32 * ch);
-            float4 *v4 = reinterpret_cast<float4 *>(p.dv32 + krow * HD + 32 * ch);
+        const int64_t trow = x.slab * p.rows + (int64_t)x.T * BK + r;
+        const float *share = nullptr;          // the block's 1/B share of a pooled gradient
+        if (p.qmajor) {
+            // dQ of query tile T + its block's share of dq̄
+            share = p.dqbar + (x.slab * p.m_pad + x.tb) * HD + 32 * ch;
+            store_row32_bf16(p.dq + trow * HD + 32 * ch, dk, share, p.inv_block);
+        } else if (p.dense) {
+            float4 *k4 = reinterpret_cast<float4 *>(p.dk32 + trow * HD + 32 * ch);
+            float4 *v4 = reinterpret_cast<float4 *>(p.dv32 + trow * HD + 32 * ch);
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 k4[e] = make_float4(dk[4 * e], dk[4 * e + 1], dk[4 * e + 2], dk[4 * e + 3]);
                 v4[e] = make_float4(dv[4 * e], dv[4 * e + 1], dv[4 * e + 2], dv[4 * e + 3]);
             }
         } else {
-            // + the key block's 1/B share of the pooled gradients dk̄_J, dv̄_J
-            const float *kb = p.dkbar + (x.slab * p.m_pad + x.jb) * HD + 32 * ch;
-            const float *vb = p.dvbar + (x.slab * p.m_pad + x.jb) * HD + 32 * ch;
-            uint4 *k4 = reinterpret_cast<uint4 *>(p.dk + krow * HD + 32 * ch);
-            uint4 *v4 = reinterpret_cast<uint4 *>(p.dv + krow * HD + 32 * ch);
-            const float ib = p.inv_block;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                uint32_t wk[4], wv[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int cc = 8 * e + 2 * h;
-                    wk[h] = pack_bf16x2(fmaf(__ldg(kb + cc), ib, dk[cc]), fmaf(__ldg(kb + cc + 1), ib, dk[cc + 1]));
-                    wv[h] = pack_bf16x2(fmaf(__ldg(vb + cc), ib, dv[cc]), fmaf(__ldg(vb + cc + 1), ib, dv[cc + 1]));
-                }
-                k4[e] = make_uint4(wk[0], wk[1], wk[2], wk[3]);
-                v4[e] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-            }
+            // dK, dV of key tile T + its block's shares of dk̄, dv̄
+            share = p.dkbar + (x.slab * p.m_pad + x.tb) * HD + 32 * ch;
+            store_row32_bf16(p.dk + trow * HD + 32 * ch, dk, share, p.inv_block);
+            share = p.dvbar + (x.slab * p.m_pad + x.tb) * HD + 32 * ch;
+            store_row32_bf16(p.dv + trow * HD + 32 * ch, dv, share, p.inv_block);
         }
     }
 }
@@ -429,10 +515,10 @@ attend_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
         for (int q = 0; q < NPIPE; ++q) {
             PipeBars &B = sh.bars[q];
             for (int b = 0; b < 2; ++b) {
-                mbar_init(&B.kv_full[b], 1);
-                mbar_init(&B.kv_empty[b], 1);
-                mbar_init(&B.qo_full[b], 1);
-                mbar_init(&B.qo_empty[b], 1);
+                mbar_init(&B.ut_full[b], 1);
+                mbar_init(&B.ut_empty[b], 1);
+                mbar_init(&B.st_full[b], 1);
+                mbar_init(&B.st_empty[b], 1);
                 mbar_init(&B.ds_full[b], 128);
                 mbar_init(&B.ds_empty[b], 1);
             }
@@ -457,12 +543,16 @@ attend_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
     __syncthreads();
     fence_after();
     const uint32_t tmem = sh.tmem_base;
-    if (warp < NPIPE) {
-        mma_role(p, sh.tiles[warp], sh.bars[warp], tmem, warp, abort_flag);
-    } else if (warp < 2 * NPIPE) {
-        const int q = warp - NPIPE;
-        loader_role(p, &tq, &tk, &tv, &to, sh.tiles[q], sh.bars[q], q, abort_flag);
+    if (warp < 2 * NPIPE) {
+        if constexpr (NPIPE == 3) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
+        if (warp < NPIPE) {
+            mma_role(p, sh.tiles[warp], sh.bars[warp], tmem, warp, abort_flag);
+        } else {
+            const int q = warp - NPIPE;
+            loader_role(p, &tq, &tk, &tv, &to, sh.tiles[q], sh.bars[q], q, abort_flag);
+        }
     } else {
+        if constexpr (NPIPE == 3) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
         const int q = (warp - 2 * NPIPE) >> 2;
         softmax_role(p, sh.tiles[q], sh.bars[q], tmem, q, warp & 3, lane, abort_flag);
     }
@@ -491,6 +581,12 @@ cudaError_t launch(const BwdParams &p, const void *q, const void *k, const void 
     const size_t smem = sizeof(SharedStorage) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attend_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    if (NPIPE == 3) {   // the register split must fit the registers the CTA is launched with
+        cudaFuncAttributes fa;
+        if ((e = cudaFuncGetAttributes(&fa, attend_bwd_tc_kernel)) != cudaSuccess) return e;
+        if ((int64_t)fa.numRegs * NTHREADS < kRegsNeeded || fa.maxThreadsPerBlock < NTHREADS)
+            return cudaErrorInvalidConfiguration;
+    }
     attend_bwd_tc_kernel<<<grid, NTHREADS, smem, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
@@ -520,6 +616,7 @@ cudaError_t launch_attend_bwd_compressed(const Problem &pb, const BwdBuffers &b,
     p.valid = (int)pb.m;
     p.lse = b.lse_cg_pad;
     p.dterm = b.dcg;
+    p.with_dq = 1;
     p.dq_acc = b.dqbar;
     p.dk32 = b.dkbar;
     p.dv32 = b.dvbar;
@@ -535,16 +632,24 @@ cudaError_t launch_attend_bwd_fine(const Problem &pb, const BwdBuffers &b, cudaS
     p.tiles = (int)(pb.n_tokens / BK);
     p.units = pb.slabs * p.tiles;
     p.valid = (int)pb.n_tokens;
-    p.offs = b.offs;
-    p.list = b.list;
     p.lse = b.lse_fine;
     p.dterm = b.dfine;
     p.gates = b.gates;
-    p.dq_acc = b.dq_acc;
-    p.dk = static_cast<__nv_bfloat16 *>(b.dk);
-    p.dv = static_cast<__nv_bfloat16 *>(b.dv);
     p.dkbar = b.dkbar;
     p.dvbar = b.dvbar;
+    p.dqbar = b.dqbar;
+    // key-major pass: dK, dV of every key tile
+    p.qmajor = 0;
+    p.offs = b.offs;
+    p.list = b.list;
+    p.dk = static_cast<__nv_bfloat16 *>(b.dk);
+    p.dv = static_cast<__nv_bfloat16 *>(b.dv);
+    cudaError_t e = launch(p, b.q, b.k, b.v, b.dout, pb.slabs * pb.n_tokens, stream);
+    if (e != cudaSuccess) return e;
+    // query-major pass: dQ of every query tile
+    p.qmajor = 1;
+    p.idx = b.sel_idx;
+    p.dq = static_cast<__nv_bfloat16 *>(b.dq);
     return launch(p, b.q, b.k, b.v, b.dout, pb.slabs * pb.n_tokens, stream);
 }
 

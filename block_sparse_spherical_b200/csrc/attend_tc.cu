@@ -140,7 +140,7 @@ struct TcParams {
     int64_t total_blocks;   // slabs * tiles query tiles (64 rows each)
     int64_t tiles;          // 64-row tiles per slab (N / 64)
     int m, n, w;            // blocks per slab, top-n, window (in blocks)
-    int R;                  // 64-row tiles per block (block_size / 64)
+    int R, logR;            // 64-row tiles per block (block_size / 64, a power of two) and its log2
     float scale_log2;
     int64_t withhold_v_step;   // test hook, -1 = off
 };
@@ -270,10 +270,14 @@ constexpr uint32_t kIdescPV = kIdescBase | (1u << 16);
 // is issued before P·V(t)). Step t uses the t-th selected block (t < n), then
 // the window blocks i-w .. i+w; blocks outside [0, m) are loaded as block i
 // and masked by the softmax. Selected indices are fetched two steps ahead.
+// LOGR: log2 of the 64-row tiles per block; MODE: 0 plain, 1 training outputs, 2 mirrored
+// output stores (compile-time, so that the plain forward carries none of the others' code)
+template <int LOGR>
 __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUtensorMap *tk,
                             const CUtensorMap *tv, SlotTiles &S, SlotBars &B, int slot,
                             volatile int *abort_flag) {
-    const int R = p.R, NR = p.n * R, T = (2 * p.w + 1 + p.n) * R;
+    constexpr int R = 1 << LOGR, lr = LOGR;
+    const int NR = p.n * R, T = (2 * p.w + 1 + p.n) * R;
     const int64_t stride = NSLOT * (int64_t)gridDim.x;
     uint32_t c = 0, gk = 0, gv = 0;
     uint64_t *last_bar[3] = {nullptr, nullptr, nullptr};   // Q, K, V: most recent copy
@@ -284,17 +288,18 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
         return __all_sync(0xffffffffu, wait_fast(b, par, abort_flag, p.status));
     };
     for (int64_t qi = NSLOT * (int64_t)blockIdx.x + slot; qi < p.total_blocks && ok; qi += stride, ++c) {
-        const int64_t slab = qi / p.tiles;
-        const int qt = (int)(qi - slab * p.tiles), i = qt / R;   // query tile and its block
-        const int64_t base = slab * p.n_tokens;
-        const int32_t *ix = p.idx + (slab * p.m + i) * (int64_t)p.n;
+        // query tile within its slab (a slab holds tiles = m*R tiles, so the tile's
+        // block row in idx is qi >> log2 R and its first token row is 64*qi)
+        const int qt = (int)((uint32_t)qi % (uint32_t)p.tiles), i = qt >> lr;
+        const int64_t base = (qi - qt) * BK;
+        const int32_t *ix = p.idx + (qi >> lr) * (int64_t)p.n;
         // key tile of step t: tile t%R of the (t/R)-th selected block, then of window block
         // i-w+(t-nR)/R; blocks outside [0, m) are loaded as the query tile and masked
         auto tile_of = [&](int t, int jsel) -> int {
-            const int j = t < NR ? jsel : i - p.w + (t - NR) / R;
-            return (j >= 0 && j < p.m) ? j * R + t % R : qt;
+            const int j = t < NR ? jsel : i - p.w + ((t - NR) >> lr);
+            return (j >= 0 && j < p.m) ? (j << lr) + (t & (R - 1)) : qt;
         };
-        auto sel_at = [&](int u) -> int { return u < NR ? __ldg(ix + u / R) : 0; };
+        auto sel_at = [&](int u) -> int { return u < NR ? __ldg(ix + (u >> lr)) : 0; };
         int jq[3];                          // selected blocks of steps t, t+1, t+2 (ring)
         jq[0] = sel_at(0);
         jq[1] = sel_at(1);
@@ -310,7 +315,7 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
         last_par[0] = c & 1;
         int jv = 0;                         // block of the next V copy
         auto issue_k = [&](int t, int j) -> bool {
-            if (leader && t < NR && t % R == 0 && (j < 0 || j >= p.m) && p.status)
+            if (leader && t < NR && (t & (R - 1)) == 0 && (j < 0 || j >= p.m) && p.status)
                 atomicOr(p.status, kStatusBadIndex);
             const int st = gk % NSTAGE;
             if (!wait_w(&B.k_empty[st], ((gk / NSTAGE) & 1) ^ 1)) return false;
@@ -356,9 +361,11 @@ __device__ void loader_role(const TcParams &p, const CUtensorMap *tq, const CUte
     }
 }
 
+template <int LOGR>
 __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t tmem_slot, int slot,
                          volatile int *abort_flag) {
-    const int NR = p.n * p.R, T = (2 * p.w + 1 + p.n) * p.R;
+    constexpr int R = 1 << LOGR;
+    const int NR = p.n * R, T = (2 * p.w + 1 + p.n) * R;
     const int64_t stride = NSLOT * (int64_t)gridDim.x;
     const uint32_t tS = tmem_slot + S_COL + (S_LANE << 16), tO = tmem_slot + O_COL + (O_LANE << 16);
     const uint32_t tP = tmem_slot + P_COL + (P_LANE << 16);   // P buffer b at + 32*b (P in TMEM)
@@ -429,10 +436,12 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
 
 // Softmax warpgroup of a slot. Thread (wq, lane): row r = 16*wq + lane%16,
 // columns 32*(lane/16) .. +31 of the query block's S and O.
+template <int LOGR, int MODE>
 __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t tmem_slot, int slot,
                              int wq, int lane, volatile int *abort_flag) {
     const unsigned FULL = 0xffffffffu;
-    const int R = p.R, NR = p.n * R, T = (2 * p.w + 1 + p.n) * R;
+    constexpr int R = 1 << LOGR, lr = LOGR;
+    const int NR = p.n * R, T = (2 * p.w + 1 + p.n) * R;
     const int ch = lane >> 4;              // column half of the row
     const int r = 16 * wq + (lane & 15);   // row within the query block
     const uint32_t wl = (uint32_t)(32 * wq);   // this warp's sub-partition
@@ -451,10 +460,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
         return __all_sync(FULL, mine);
     };
     // selected blocks of query tile q (its block's index row)
-    auto sel_row = [&](int64_t q) -> const int32_t * {
-        const int64_t sl = q / p.tiles;
-        return p.idx + (sl * p.m + (q - sl * p.tiles) / R) * (int64_t)p.n;
-    };
+    auto sel_row = [&](int64_t q) -> const int32_t * { return p.idx + (q >> lr) * (int64_t)p.n; };
     int j0 = 0, j1 = 0;                    // this lane's two selected indices of the next query tile
     {
         const int64_t q0 = NSLOT * (int64_t)blockIdx.x + slot;
@@ -465,12 +471,11 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
         }
     }
     for (int64_t qi = NSLOT * (int64_t)blockIdx.x + slot; qi < p.total_blocks && ok; qi += stride) {
-        const int64_t slab = qi / p.tiles;
-        const int qt = (int)(qi - slab * p.tiles), i = qt / R;   // query tile and its block
-        const int64_t tok = slab * p.n_tokens + (int64_t)qt * BK + r;
+        const int qt = (int)((uint32_t)qi % (uint32_t)p.tiles), i = qt >> lr;   // tile within the slab, its block
+        const int64_t tok = qi * BK + r;
         const float *gp = p.gates + tok * 3;
         const float g_cg = __ldg(gp), g_fg = __ldg(gp + 1), g_l = __ldg(gp + 2);
-        const float *ocg = p.o_cg + (slab * p.m + i) * (int64_t)HD + 32 * ch;
+        const float *ocg = p.o_cg + (qi >> lr) * (int64_t)HD + 32 * ch;
         asm volatile("prefetch.global.L1 [%0];" ::"l"(ocg));
         // validity of the n selected blocks of this query block, as a bit mask
         // (its indices were fetched during the previous query block)
@@ -490,9 +495,9 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
         for (int t = 0; t < T; ++t, ++g) {
             bool valid;
             if (t < NR) {
-                valid = (selmask >> (t / R)) & 1u;
+                valid = (selmask >> (t >> lr)) & 1u;
             } else {
-                const int j = i - p.w + (t - NR) / R;
+                const int j = i - p.w + ((t - NR) >> lr);
                 valid = j >= 0 && j < p.m;
             }
             if (t == NR) {                     // the local branch starts afresh
@@ -551,7 +556,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 tmem_ld16(tO, a);
                 tmem_ld16(tO + 16, a + 16);
                 tmem_wait_ld();
-                if (p.o_fg) {                  // training: o_FG and its row log-sum-exp
+                if constexpr (MODE == 1) {     // training: o_FG and its row log-sum-exp
                     const float inv1 = l > 0.f ? 1.f / l : 0.f;
                     store_row32(p.o_fg + tok * HD + 32 * ch, a, inv1);
                     if (ch == 0) p.lse[tok * 2] = (m_sel + __log2f(l)) * 0.69314718055994531f;
@@ -604,7 +609,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
         fence_after();
         const float l = l_run + __shfl_xor_sync(FULL, l_run, 16);
         const float inv = l > 0.f ? g_l / l : 0.f;
-        if (p.o_l) {                           // training: o_L and its row log-sum-exp
+        if constexpr (MODE == 1) {             // training: o_L and its row log-sum-exp
             float o[32];
             tmem_ld16(tO, o);
             tmem_ld16(tO + 16, o + 16);
@@ -626,16 +631,19 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             const uint4 lo4 = make_uint4(w8[0], w8[1], w8[2], w8[3]), hi4 = make_uint4(w8[4], w8[5], w8[6], w8[7]);
             d4[2 * cc] = lo4;
             d4[2 * cc + 1] = hi4;
-            for (int mi = 0; mi < p.n_mirror; ++mi) {
-                uint4 *m4 = reinterpret_cast<uint4 *>(p.mirror[mi] + tok * HD + 32 * ch);
-                m4[2 * cc] = lo4;
-                m4[2 * cc + 1] = hi4;
+            if constexpr (MODE == 2) {
+                for (int mi = 0; mi < p.n_mirror; ++mi) {
+                    uint4 *m4 = reinterpret_cast<uint4 *>(p.mirror[mi] + tok * HD + 32 * ch);
+                    m4[2 * cc] = lo4;
+                    m4[2 * cc + 1] = hi4;
+                }
             }
         }
         fence_before();
     }
 }
 
+template <int LOGR, int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                  const __grid_constant__ CUtensorMap tv, const TcParams p) {
@@ -686,13 +694,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
         const int slot = warp % NSLOT;
         if (warp < NSLOT)
-            mma_role(p, sh.tiles[slot], sh.bars[slot], tmem + 128u * slot, slot, abort_flag);
+            mma_role<LOGR>(p, sh.tiles[slot], sh.bars[slot], tmem + 128u * slot, slot, abort_flag);
         else
-            loader_role(p, &tq, &tk, &tv, sh.tiles[slot], sh.bars[slot], slot, abort_flag);
+            loader_role<LOGR>(p, &tq, &tk, &tv, sh.tiles[slot], sh.bars[slot], slot, abort_flag);
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
         const int slot = (warp - 2 * NSLOT) >> 2;
-        softmax_role(p, sh.tiles[slot], sh.bars[slot], tmem + 128u * slot, slot, warp & 3, lane, abort_flag);
+        softmax_role<LOGR, MODE>(p, sh.tiles[slot], sh.bars[slot], tmem + 128u * slot, slot, warp & 3, lane,
+                                 abort_flag);
     }
     __syncwarp();                          // reconverge role lanes before the CTA barrier
 
@@ -720,6 +729,24 @@ __global__ void exp2_eval_kernel(const float *__restrict__ x, float *__restrict_
         y[i] = e.x;
         if (i + 1 < n) y[i + 1] = e.y;
     }
+}
+
+template <int LOGR, int MODE>
+cudaError_t launch_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const TcParams &p,
+                          int grid, cudaStream_t stream) {
+    auto kern = attend_tc_kernel<LOGR, MODE>;
+    const size_t smem = sizeof(SharedStorage) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // The register split must fit the registers the CTA is launched with,
+    // otherwise setmaxnreg.inc would wait forever: refuse to launch instead.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if ((int64_t)fa.numRegs * NTHREADS < kRegsNeeded || fa.maxThreadsPerBlock < NTHREADS)
+        return cudaErrorInvalidConfiguration;
+    kern<<<grid, NTHREADS, smem, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -759,6 +786,9 @@ cudaError_t launch_attend_tc(const Problem &pb, const void *q, const void *k, co
     p.n = (int)pb.top_n;
     p.w = (int)pb.window;
     p.R = (int)(pb.block_size / BK);
+    p.logR = 0;
+    while ((1 << p.logR) < p.R) ++p.logR;
+    if ((1 << p.logR) != p.R) return cudaErrorNotSupported;   // blocks of 64 * 2^k tokens
     p.tiles = pb.n_tokens / BK;
     p.total_blocks = pb.slabs * p.tiles;
     p.scale_log2 = pb.scale * 1.4426950408889634f;
@@ -767,18 +797,20 @@ cudaError_t launch_attend_tc(const Problem &pb, const void *q, const void *k, co
     if (sms <= 0) return cudaErrorInvalidDevice;
     const int64_t want = (p.total_blocks + NSLOT - 1) / NSLOT;
     const int grid = (int)(want < sms ? want : sms);
-    const size_t smem = sizeof(SharedStorage) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    // The register split must fit the registers the CTA is launched with,
-    // otherwise setmaxnreg.inc would wait forever: refuse to launch instead.
-    cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, attend_tc_kernel);
-    if (e != cudaSuccess) return e;
-    if ((int64_t)fa.numRegs * NTHREADS < kRegsNeeded || fa.maxThreadsPerBlock < NTHREADS)
-        return cudaErrorInvalidConfiguration;
-    attend_tc_kernel<<<grid, NTHREADS, smem, stream>>>(tq, tk, tv, p);
-    return cudaGetLastError();
+    if (p.o_fg && n_mirrors > 0) return cudaErrorInvalidValue;   // one extra output kind per launch
+    const int mode = p.o_fg ? 1 : (n_mirrors > 0 ? 2 : 0);
+    switch (p.logR * 3 + mode) {
+        case 0: return launch_kernel<0, 0>(tq, tk, tv, p, grid, stream);
+        case 1: return launch_kernel<0, 1>(tq, tk, tv, p, grid, stream);
+        case 2: return launch_kernel<0, 2>(tq, tk, tv, p, grid, stream);
+        case 6: return launch_kernel<2, 0>(tq, tk, tv, p, grid, stream);
+        case 7: return launch_kernel<2, 1>(tq, tk, tv, p, grid, stream);
+        case 8: return launch_kernel<2, 2>(tq, tk, tv, p, grid, stream);
+        case 12: return launch_kernel<4, 0>(tq, tk, tv, p, grid, stream);
+        case 13: return launch_kernel<4, 1>(tq, tk, tv, p, grid, stream);
+        case 14: return launch_kernel<4, 2>(tq, tk, tv, p, grid, stream);
+        default: return cudaErrorNotSupported;   // blocks of 64, 256 or 1024 tokens
+    }
 }
 
 }  // namespace bsa

@@ -14,8 +14,6 @@
 //                     tensor-core pass over the compressed branch
 //   inv_*_kernel      the selection inverted: for every key block j the query
 //                     blocks i whose top-n holds j, ascending (CSR per slab)
-//   bwd_finalize_dq   dq_t = dq_acc_t + dq̄_i / B (the mean hands each token of
-//                     block i a 1/B share of the pooled gradient), as bf16
 #include <math_constants.h>
 
 #include "bsa_internal.cuh"
@@ -191,24 +189,6 @@ __global__ void inv_sort_kernel(const int *__restrict__ offs, const int *__restr
     }
 }
 
-// dq_t = bf16(dq_acc_t + dq̄_{i(t)} / B), four channels a thread.
-__global__ void bwd_finalize_dq_kernel(const float *__restrict__ dq_acc, const float *__restrict__ dqbar,
-                                       __nv_bfloat16 *__restrict__ dq, int64_t rows, int64_t n_tokens, int m_pad,
-                                       int block, float inv_block) {
-    const int64_t total = rows * (HD / 4);
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t row = e / (HD / 4);
-        const int c4 = (int)(e - row * (HD / 4));
-        const int64_t slab = row / n_tokens;
-        const int i = (int)((row - slab * n_tokens) / block);
-        const float4 a = *reinterpret_cast<const float4 *>(dq_acc + row * HD + 4 * c4);
-        const float4 b = *reinterpret_cast<const float4 *>(dqbar + (slab * m_pad + i) * HD + 4 * c4);
-        __nv_bfloat162 *d = reinterpret_cast<__nv_bfloat162 *>(dq + row * HD + 4 * c4);
-        d[0] = __floats2bfloat162_rn(fmaf(b.x, inv_block, a.x), fmaf(b.y, inv_block, a.y));
-        d[1] = __floats2bfloat162_rn(fmaf(b.z, inv_block, a.z), fmaf(b.w, inv_block, a.w));
-    }
-}
-
 int grid_for(int64_t work, int threads) {
     const int64_t g = (work + threads - 1) / threads;
     return (int)(g < 148 * 16 ? (g > 0 ? g : 1) : 148 * 16);
@@ -240,15 +220,6 @@ cudaError_t launch_inverse_index(const Problem &p, const int32_t *idx, int *coun
     const int64_t warps = p.slabs * p.m;
     inv_sort_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, stream>>>(offs, list_tmp, list, (int)p.m,
                                                                              (int)p.top_n, warps);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_bwd_finalize_dq(const Problem &p, const float *dq_acc, const float *dqbar, int64_t m_pad,
-                                   void *dq, cudaStream_t stream) {
-    const int64_t rows = p.slabs * p.n_tokens;
-    bwd_finalize_dq_kernel<<<grid_for(rows * (HD / 4), 256), 256, 0, stream>>>(
-        dq_acc, dqbar, static_cast<__nv_bfloat16 *>(dq), rows, p.n_tokens, (int)m_pad, (int)p.block_size,
-        1.f / (float)p.block_size);
     return cudaGetLastError();
 }
 

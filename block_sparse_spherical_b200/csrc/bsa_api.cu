@@ -201,7 +201,7 @@ namespace {
 bool train_supported(const Problem &p) { return p.dtype == BSA_BF16 && p.head_dim == 64; }
 
 struct BwdLayout {
-    size_t status, qbar, kbar, vbar, dfine, docg16, q16, k16, v16, dcg, lse_pad, dqbar, dkbar, dvbar, dq_acc;
+    size_t status, qbar, kbar, vbar, dfine, docg16, q16, k16, v16, dcg, lse_pad, dqbar, dkbar, dvbar;
     size_t count, offs, cursor, list_tmp, list, total;
     int64_t m_pad;
 };
@@ -230,7 +230,6 @@ BwdLayout bwd_layout_of(const Problem &p) {
     L.dqbar = take(pad32);
     L.dkbar = take(pad32);
     L.dvbar = take(pad32);
-    L.dq_acc = take(rows * p.head_dim * sizeof(float));
     L.count = take(ints_m);
     L.offs = take((size_t)p.slabs * (p.m + 1) * sizeof(int));
     L.cursor = take(ints_m);
@@ -323,23 +322,20 @@ bsa_status bsa_backward(const bsa_config *cfg, const void *q, const void *k, con
     b.dqbar = reinterpret_cast<float *>(ws + L.dqbar);
     b.dkbar = reinterpret_cast<float *>(ws + L.dkbar);
     b.dvbar = reinterpret_cast<float *>(ws + L.dvbar);
-    b.dq_acc = reinterpret_cast<float *>(ws + L.dq_acc);
     b.count = reinterpret_cast<int *>(ws + L.count);
     b.offs = reinterpret_cast<int *>(ws + L.offs);
     b.cursor = reinterpret_cast<int *>(ws + L.cursor);
     b.list_tmp = reinterpret_cast<int *>(ws + L.list_tmp);
     b.list = reinterpret_cast<int *>(ws + L.list);
-    // the two gradient accumulators start at zero (memsets, not allocations)
-    cudaError_t e = cudaMemsetAsync(ws + L.dq_acc, 0, (size_t)p.slabs * p.n_tokens * p.head_dim * sizeof(float),
-                                    stream);
-    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.dqbar, 0, (size_t)p.slabs * L.m_pad * p.head_dim * 4, stream);
+    // the pooled dq̄ is reduced into from every key tile of the compressed pass: it starts at zero
+    // (a memset, not an allocation)
+    cudaError_t e = cudaMemsetAsync(ws + L.dqbar, 0, (size_t)p.slabs * L.m_pad * p.head_dim * 4, stream);
     if (e == cudaSuccess) e = bsa::launch_pool(p, q, k, v, b.qbar, b.kbar, b.vbar, stream);
     if (e == cudaSuccess) e = bsa::launch_bwd_prep(p, b, stream);
     if (e == cudaSuccess) e = bsa::launch_attend_bwd_compressed(p, b, stream);
     if (e == cudaSuccess)
         e = bsa::launch_inverse_index(p, sel_idx, b.count, b.offs, b.cursor, b.list_tmp, b.list, b.status, stream);
-    if (e == cudaSuccess) e = bsa::launch_attend_bwd_fine(p, b, stream);
-    if (e == cudaSuccess) e = bsa::launch_bwd_finalize_dq(p, b.dq_acc, b.dqbar, L.m_pad, dq, stream);
+    if (e == cudaSuccess) e = bsa::launch_attend_bwd_fine(p, b, stream);   // dk, dv, then dq
     return from_cuda(e);
 }
 
@@ -366,21 +362,28 @@ bsa_status bsa_latlon_healpix_plan(int64_t nside, int64_t nlat, int64_t nlon, in
     return from_cuda(bsa::launch_healpix_plan(nside, nlat, nlon, nbr, rel, stream));
 }
 
+bsa_status bsa_latlon_workspace_size(int64_t batch, int64_t n_src, size_t *bytes) {
+    if (batch < 1 || n_src < 1 || !bytes) return BSA_ERR_INVALID_ARG;
+    *bytes = round_up((size_t)batch * n_src * 3 * sizeof(float));
+    return BSA_OK;
+}
+
 bsa_status bsa_latlon_to_healpix(int64_t batch, int64_t n_tgt, int64_t n_src, int64_t head_dim, int32_t dtype,
                                  float scale, const int32_t *nbr, const float *rel, const float *wq,
-                                 const void *k_src, const void *v_src, void *out, uint32_t *status_word,
-                                 cudaStream_t stream) {
+                                 const void *k_src, const void *v_src, void *out, void *workspace,
+                                 size_t workspace_bytes, uint32_t *status_word, cudaStream_t stream) {
     if (batch < 1 || batch > 65535 || n_tgt < 1 || n_src < 1 || n_src > 0x7fffffffLL) return BSA_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < (size_t)batch * n_src * 3 * sizeof(float)) return BSA_ERR_WORKSPACE;
     if (dtype != BSA_F32 && dtype != BSA_BF16) return BSA_ERR_INVALID_ARG;
     if (!(scale >= 0.0f) || isinf(scale)) return BSA_ERR_INVALID_ARG;
     if (head_dim != 32 && head_dim != 64 && head_dim != 128) return BSA_ERR_UNSUPPORTED;
     if (!nbr || !rel || !wq || !k_src || !v_src || !out) return BSA_ERR_INVALID_ARG;
     if (!aligned16(nbr) || !aligned16(rel) || !aligned16(wq) || !aligned16(k_src) || !aligned16(v_src) ||
-        !aligned16(out) || ((uintptr_t)status_word & 3u))
+        !aligned16(out) || !aligned16(workspace) || ((uintptr_t)status_word & 3u))
         return BSA_ERR_ALIGNMENT;
     const float s = scale > 0.0f ? scale : 1.0f / sqrtf((float)head_dim);
     return from_cuda(bsa::launch_interp(batch, n_tgt, n_src, head_dim, (bsa_dtype)dtype, nbr, rel, wq, k_src, v_src,
-                                        out, s, status_word, stream));
+                                        out, s, static_cast<float *>(workspace), status_word, stream));
 }
 
 bsa_status bsa_forward_mirrored(const bsa_config *cfg, const void *q, const void *k, const void *v,

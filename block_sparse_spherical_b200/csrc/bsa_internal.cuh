@@ -68,7 +68,7 @@ cudaError_t launch_healpix_plan(int64_t nside, int64_t nlat, int64_t nlon, int32
                                 cudaStream_t stream);
 cudaError_t launch_interp(int64_t batch, int64_t n_tgt, int64_t n_src, int64_t d, bsa_dtype dtype,
                           const int32_t *nbr, const float *rel, const float *wq, const void *k, const void *v,
-                          void *out, float scale, uint32_t *status, cudaStream_t stream);
+                          void *out, float scale, float *kappa, uint32_t *status, cudaStream_t stream);
 
 // Test hook: the fine-attention kernel's exp2 on the FMA pipe (poly != 0) or the exp unit.
 cudaError_t launch_exp2_eval(const float *x, float *y, int64_t n, int poly, cudaStream_t stream);
@@ -96,17 +96,15 @@ struct BwdBuffers {
     void *docg16, *q16, *k16, *v16; // [slabs*m_pad][64] bf16 (zero rows past m)
     float *dcg, *lse_cg_pad;        // [slabs*m_pad]
     float *dqbar, *dkbar, *dvbar;   // [slabs*m_pad][64]: gradients of q̄, k̄, v̄
-    float *dq_acc;                  // [slabs*N][64]
     int *count, *offs, *cursor, *list_tmp, *list;   // the inverted selection
 };
 cudaError_t launch_bwd_prep(const Problem &p, const BwdBuffers &b, cudaStream_t stream);
 cudaError_t launch_inverse_index(const Problem &p, const int32_t *idx, int *count, int *offs, int *cursor,
                                  int *list_tmp, int *list, uint32_t *status, cudaStream_t stream);
-cudaError_t launch_bwd_finalize_dq(const Problem &p, const float *dq_acc, const float *dqbar, int64_t m_pad,
-                                   void *dq, cudaStream_t stream);
-// Attention backward on the tensor cores, by key tile: the compressed branch
-// (dense over the 64-block tiles of q̄, k̄, v̄, dO_CG) or the two fine branches
-// (each key block's window and the query blocks that selected it).
+// Attention backward on the tensor cores: the compressed branch (by key tile, dense
+// over the 64-block tiles of q̄, k̄, v̄, dO_CG; dq̄ reduced into b.dqbar) and the two
+// fine branches (dk, dv by key tile over each key block's window and the query
+// blocks that selected it; then dq by query tile over its selected and window blocks).
 cudaError_t launch_attend_bwd_compressed(const Problem &p, const BwdBuffers &b, cudaStream_t stream);
 cudaError_t launch_attend_bwd_fine(const Problem &p, const BwdBuffers &b, cudaStream_t stream);
 

@@ -61,7 +61,7 @@ constexpr uint32_t TMEM_COLS = 256;        // S buffers at columns 0 and 64, O b
 // two warpgroups drop to kCtlRegs. 128·kRowRegs + 256·kCtlRegs must not exceed
 // 384·168 (the host checks the compiled launch count), or setmaxnreg.inc would
 // wait forever.
-constexpr int kRowRegs = 232, kCtlRegs = 136;
+constexpr int kRowRegs = 240, kCtlRegs = 128;
 constexpr int kRegsNeeded = 128 * kRowRegs + 256 * kCtlRegs;
 
 // instruction descriptor: D f32, A and B tf32, both K-major, M = 128, N = 64

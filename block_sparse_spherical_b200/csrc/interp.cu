@@ -10,11 +10,13 @@
 //   r0..r0+3, r0 = floor((90 - lat)/dlat) - 1 clamped to [0, nlat-4]; columns
 //   c0-1..c0+2 wrapping in longitude, c0 = floor(lon/dlon)) and the relative
 //   positions (x_j - x_i)/dlat_rad. The integer decisions use fp64.
-// interp_kernel: one warp per target: lane l holds channels l*C..l*C+C-1
-//   (C = d/32); per neighbour the query channels W_q p_ij, a warp-reduced dot
-//   with k_j, then an exact softmax over the 16 logits and the weighted sum
-//   of the v_j rows, which are gathered from the small (L2-resident) source
-//   grid. fp32 arithmetic; bf16 or fp32 features.
+// kappa_kernel + interp_kernel: (W_q p_ij)·k_j = p_ij·(W_qᵀ k_j), so every
+//   source key is first reduced to kappa_j = W_qᵀ k_j (3 floats, once per source
+//   point, into the caller's workspace); then one half-warp per target, lane j
+//   holding neighbour j: logit p_ij·kappa_j, exact softmax over the 16 lanes,
+//   and each lane sums d/16 channels of the v_j rows gathered from the small
+//   (L2-resident) source grid; the batch loops inside, so the plan is read
+//   once. fp32 arithmetic; bf16 or fp32 features.
 #include "bsa_internal.cuh"
 
 namespace bsa {
@@ -84,89 +86,119 @@ template <> __device__ __forceinline__ float load1<__nv_bfloat16>(const __nv_bfl
     return __bfloat162float(*p);
 }
 
+// kappa[b][j][e] = s·log2(e) · Σ_c W_q[c][e] k[b][j][c]: each source key seen from position
+// space, so that the logit of (i, j) is p_ij · kappa_j (= s (W_q p_ij)·k_j). One warp per source
+// point, lane l holding channels l*C .. l*C+C-1.
 template <typename T, int C>
 __global__ void __launch_bounds__(256)
-interp_kernel(int64_t n_tgt, int64_t n_src, const int32_t *__restrict__ nbr, const float *__restrict__ rel,
-              const float *__restrict__ wq, const T *__restrict__ ksrc, const T *__restrict__ vsrc,
-              T *__restrict__ out, float scale_log2, uint32_t *status) {
+kappa_kernel(int64_t rows, const float *__restrict__ wq, const T *__restrict__ ksrc, float *__restrict__ kappa,
+             float scale_log2) {
     constexpr int D = 32 * C;
     const int lane = threadIdx.x & 31;
-    const int64_t batch = blockIdx.y;
-    const T *kb = ksrc + batch * n_src * D, *vb = vsrc + batch * n_src * D;
     float w[C][3];
 #pragma unroll
     for (int c = 0; c < C; ++c)
 #pragma unroll
         for (int e = 0; e < 3; ++e) w[c][e] = __ldg(wq + (lane * C + c) * 3 + e);
-    for (int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; i < n_tgt;
-         i += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-        int32_t src[KN];
-        float lg[KN];
-        bool bad = false;
+    for (int64_t r = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; r < rows;
+         r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f;
 #pragma unroll
-        for (int j = 0; j < KN; ++j) {
-            src[j] = __ldg(nbr + i * KN + j);
-            if (src[j] < 0 || src[j] >= n_src) {
-                bad = true;
-                src[j] = 0;
+        for (int c = 0; c < C; ++c) {
+            const float kc = load1<T>(ksrc + r * D + lane * C + c);
+            a0 = fmaf(w[c][0], kc, a0);
+            a1 = fmaf(w[c][1], kc, a1);
+            a2 = fmaf(w[c][2], kc, a2);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            a0 += __shfl_xor_sync(0xffffffffu, a0, off);
+            a1 += __shfl_xor_sync(0xffffffffu, a1, off);
+            a2 += __shfl_xor_sync(0xffffffffu, a2, off);
+        }
+        if (lane == 0) {
+            kappa[r * 3] = a0 * scale_log2;
+            kappa[r * 3 + 1] = a1 * scale_log2;
+            kappa[r * 3 + 2] = a2 * scale_log2;
+        }
+    }
+}
+
+// One half-warp per target pixel, all batch elements in turn (the plan is read once).
+// Lane j of the half holds neighbour j: its logit p_ij·kappa_j (log2 domain), then the
+// softmax over the 16 lanes; each lane then sums C4 = d/16 channels of Σ_j p_j v_j.
+template <typename T, int C4>
+__global__ void __launch_bounds__(256)
+interp_kernel(int64_t batch, int64_t n_tgt, int64_t n_src, const int32_t *__restrict__ nbr,
+              const float *__restrict__ rel, const float *__restrict__ kappa, const T *__restrict__ vsrc,
+              T *__restrict__ out, uint32_t *status) {
+    constexpr int D = 16 * C4;
+    const int lane = threadIdx.x & 31, j = lane & 15;
+    const unsigned half = (lane < 16) ? 0x0000ffffu : 0xffff0000u;
+    const int64_t halves = ((int64_t)gridDim.x * blockDim.x) >> 4;
+    for (int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 4; i < n_tgt; i += halves) {
+        int32_t src = __ldg(nbr + i * KN + j);
+        const bool bad = src < 0 || src >= n_src;
+        if (bad) src = 0;
+        const float *pr = rel + (i * KN + j) * 3;
+        const float p0 = __ldg(pr), p1 = __ldg(pr + 1), p2 = __ldg(pr + 2);
+        if (__any_sync(half, bad) && j == 0 && status) atomicOr(status, kStatusBadIndex);
+        for (int64_t b = 0; b < batch; ++b) {
+            const float *kp = kappa + (b * n_src + src) * 3;
+            float lg = fmaf(p0, __ldg(kp), fmaf(p1, __ldg(kp + 1), p2 * __ldg(kp + 2)));
+            float mx = lg;
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(half, mx, off));
+            const float e = exp2f(lg - mx);
+            float den = e;
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) den += __shfl_xor_sync(half, den, off);
+            const float pj = e / den;
+            float acc[C4];
+#pragma unroll
+            for (int c = 0; c < C4; ++c) acc[c] = 0.f;
+            const T *vb = vsrc + b * n_src * D;
+#pragma unroll
+            for (int jj = 0; jj < KN; ++jj) {
+                const float pw = __shfl_sync(half, pj, (lane & 16) | jj);
+                const int32_t sj = __shfl_sync(half, src, (lane & 16) | jj);
+                const T *vr = vb + (int64_t)sj * D + j * C4;
+#pragma unroll
+                for (int c = 0; c < C4; ++c) acc[c] = fmaf(pw, load1<T>(vr + c), acc[c]);
             }
+            T *o = out + (b * n_tgt + i) * D + j * C4;
+#pragma unroll
+            for (int c = 0; c < C4; ++c) o[c] = from_f32<T>(acc[c]);
         }
-#pragma unroll
-        for (int j = 0; j < KN; ++j) {
-            const float *pr = rel + (i * KN + j) * 3;
-            const float p0 = __ldg(pr), p1 = __ldg(pr + 1), p2 = __ldg(pr + 2);
-            const T *kr = kb + (int64_t)src[j] * D + lane * C;
-            float part = 0.f;
-#pragma unroll
-            for (int c = 0; c < C; ++c) {
-                const float qc = fmaf(w[c][0], p0, fmaf(w[c][1], p1, w[c][2] * p2));
-                part = fmaf(qc, load1<T>(kr + c), part);
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-            lg[j] = part * scale_log2;      // log2 domain
-        }
-        float mx = lg[0];
-#pragma unroll
-        for (int j = 1; j < KN; ++j) mx = fmaxf(mx, lg[j]);
-        float den = 0.f;
-#pragma unroll
-        for (int j = 0; j < KN; ++j) {
-            lg[j] = exp2f(lg[j] - mx);
-            den += lg[j];
-        }
-        const float inv = 1.f / den;
-        float acc[C];
-#pragma unroll
-        for (int c = 0; c < C; ++c) acc[c] = 0.f;
-#pragma unroll
-        for (int j = 0; j < KN; ++j) {
-            const T *vr = vb + (int64_t)src[j] * D + lane * C;
-#pragma unroll
-            for (int c = 0; c < C; ++c) acc[c] = fmaf(lg[j], load1<T>(vr + c), acc[c]);
-        }
-        T *o = out + (batch * n_tgt + i) * D + lane * C;
-#pragma unroll
-        for (int c = 0; c < C; ++c) o[c] = from_f32<T>(acc[c] * inv);
-        if (bad && lane == 0 && status) atomicOr(status, kStatusBadIndex);
     }
 }
 
 template <typename T>
 cudaError_t launch_interp_t(int64_t batch, int64_t n_tgt, int64_t n_src, int64_t d, const int32_t *nbr,
                             const float *rel, const float *wq, const void *k, const void *v, void *out, float scale,
-                            uint32_t *status, cudaStream_t stream) {
-    int64_t ctas = (n_tgt * 32 + 255) / 256;
-    if (ctas > 148 * 64) ctas = 148 * 64;
-    if (ctas < 1) ctas = 1;
-    const dim3 grid((unsigned)ctas, (unsigned)batch);
+                            float *kappa, uint32_t *status, cudaStream_t stream) {
     const float sl2 = scale * 1.4426950408889634f;
     const T *kt = static_cast<const T *>(k), *vt = static_cast<const T *>(v);
     T *ot = static_cast<T *>(out);
+    const int64_t krows = batch * n_src;
+    int64_t kctas = (krows * 32 + 255) / 256;
+    if (kctas > 148 * 32) kctas = 148 * 32;
+    int64_t ctas = (n_tgt * 16 + 255) / 256;
+    if (ctas > 148 * 64) ctas = 148 * 64;
+    if (ctas < 1) ctas = 1;
     switch (d) {
-        case 32: interp_kernel<T, 1><<<grid, 256, 0, stream>>>(n_tgt, n_src, nbr, rel, wq, kt, vt, ot, sl2, status); break;
-        case 64: interp_kernel<T, 2><<<grid, 256, 0, stream>>>(n_tgt, n_src, nbr, rel, wq, kt, vt, ot, sl2, status); break;
-        case 128: interp_kernel<T, 4><<<grid, 256, 0, stream>>>(n_tgt, n_src, nbr, rel, wq, kt, vt, ot, sl2, status); break;
+        case 32:
+            kappa_kernel<T, 1><<<(unsigned)kctas, 256, 0, stream>>>(krows, wq, kt, kappa, sl2);
+            interp_kernel<T, 2><<<(unsigned)ctas, 256, 0, stream>>>(batch, n_tgt, n_src, nbr, rel, kappa, vt, ot, status);
+            break;
+        case 64:
+            kappa_kernel<T, 2><<<(unsigned)kctas, 256, 0, stream>>>(krows, wq, kt, kappa, sl2);
+            interp_kernel<T, 4><<<(unsigned)ctas, 256, 0, stream>>>(batch, n_tgt, n_src, nbr, rel, kappa, vt, ot, status);
+            break;
+        case 128:
+            kappa_kernel<T, 4><<<(unsigned)kctas, 256, 0, stream>>>(krows, wq, kt, kappa, sl2);
+            interp_kernel<T, 8><<<(unsigned)ctas, 256, 0, stream>>>(batch, n_tgt, n_src, nbr, rel, kappa, vt, ot, status);
+            break;
         default: return cudaErrorNotSupported;
     }
     return cudaGetLastError();
@@ -183,10 +215,11 @@ cudaError_t launch_healpix_plan(int64_t nside, int64_t nlat, int64_t nlon, int32
 
 cudaError_t launch_interp(int64_t batch, int64_t n_tgt, int64_t n_src, int64_t d, bsa_dtype dtype,
                           const int32_t *nbr, const float *rel, const float *wq, const void *k, const void *v,
-                          void *out, float scale, uint32_t *status, cudaStream_t stream) {
+                          void *out, float scale, float *kappa, uint32_t *status, cudaStream_t stream) {
     if (dtype == BSA_BF16)
-        return launch_interp_t<__nv_bfloat16>(batch, n_tgt, n_src, d, nbr, rel, wq, k, v, out, scale, status, stream);
-    return launch_interp_t<float>(batch, n_tgt, n_src, d, nbr, rel, wq, k, v, out, scale, status, stream);
+        return launch_interp_t<__nv_bfloat16>(batch, n_tgt, n_src, d, nbr, rel, wq, k, v, out, scale, kappa, status,
+                                              stream);
+    return launch_interp_t<float>(batch, n_tgt, n_src, d, nbr, rel, wq, k, v, out, scale, kappa, status, stream);
 }
 
 }  // namespace bsa

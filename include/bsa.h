@@ -193,15 +193,20 @@ BSA_API bsa_status bsa_forward_mirrored(const bsa_config *cfg, const void *q, co
  * independent feature sets: k_src, v_src [batch][n_src][head_dim] and out
  * [batch][n_tgt][head_dim] in `dtype` (bf16 or fp32), wq [head_dim][3]
  * float (the query map), scale 0 = 1/sqrt(head_dim); head_dim 32, 64 or 128.
- * fp32 arithmetic. Neighbour indices outside [0, n_src) are replaced by 0 and
- * flagged BSA_ERR_INDEX in *status_word (nullable).
+ * fp32 arithmetic. The logits are formed as p_ij·(W_qᵀ k_j), the same value
+ * as (W_q p_ij)·k_j: each source key is reduced once to 3 floats, kept in
+ * `workspace` (device, 16-byte aligned, >= bsa_latlon_workspace_size bytes;
+ * BSA_ERR_WORKSPACE otherwise). Neighbour indices outside [0, n_src) are
+ * replaced by 0 and flagged BSA_ERR_INDEX in *status_word (nullable).
  */
 BSA_API bsa_status bsa_latlon_healpix_plan(int64_t nside, int64_t nlat, int64_t nlon, int32_t *nbr, float *rel,
                                            cudaStream_t stream);
+BSA_API bsa_status bsa_latlon_workspace_size(int64_t batch, int64_t n_src, size_t *bytes);
 BSA_API bsa_status bsa_latlon_to_healpix(int64_t batch, int64_t n_tgt, int64_t n_src, int64_t head_dim,
                                          int32_t dtype, float scale, const int32_t *nbr, const float *rel,
                                          const float *wq, const void *k_src, const void *v_src, void *out,
-                                         uint32_t *status_word, cudaStream_t stream);
+                                         void *workspace, size_t workspace_bytes, uint32_t *status_word,
+                                         cudaStream_t stream);
 
 /*
  * Token layouts other than HEALPix NESTED. The note's ablation "BSA but not

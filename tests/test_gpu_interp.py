@@ -78,6 +78,7 @@ def test_interp_matches_oracle(nside, nlat, nlon, d, dtype, batch):
 def test_interp_rejects_bad_arguments():
     L = abi.load()
     A = 4096
-    assert L.bsa_latlon_to_healpix(1, 10, 10, 48, 1, 0.0, A, A, A, A, A, A, None, None) == 2   # head_dim 48
-    assert L.bsa_latlon_to_healpix(1, 10, 10, 64, 5, 0.0, A, A, A, A, A, A, None, None) == 1   # dtype
+    assert L.bsa_latlon_to_healpix(1, 10, 10, 48, 1, 0.0, A, A, A, A, A, A, A, 4096, None, None) == 2   # head_dim 48
+    assert L.bsa_latlon_to_healpix(1, 10, 10, 64, 5, 0.0, A, A, A, A, A, A, A, 4096, None, None) == 1   # dtype
+    assert L.bsa_latlon_to_healpix(1, 10, 10, 64, 1, 0.0, A, A, A, A, A, A, A, 16, None, None) == 6     # workspace
     assert L.bsa_latlon_healpix_plan(3, 10, 10, A, A, None) == 1                              # nside not 2^k
