@@ -694,6 +694,9 @@ def main():
     ap.add_argument("--shard", action="store_true",
                     help="split one problem's (batch, head) slabs over the ranks (strong scaling) instead of "
                          "running an independent replica per rank")
+    ap.add_argument("--block-size", type=int, default=None,
+                    help="override the workload's block size (tokens per block: 64, 256 or 1024 for bf16)")
+    ap.add_argument("--top-n", type=int, default=None, help="override the workload's top-n")
     ap.add_argument("--fused-gather", action="store_true",
                     help="with --shard: the kernel's epilogue stores output rows into every rank's buffer "
                          "(symmetric memory) instead of an NCCL all-gather after the forward")
@@ -704,6 +707,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     cfg = CONFIGS[args.workload]
+    if args.block_size or args.top_n:
+        bk = args.block_size or cfg.block_size
+        cfg = cfg.with_(name=f"{cfg.name}_block{bk}_n{args.top_n or cfg.top_n}", block_size=bk,
+                        top_n=args.top_n or cfg.top_n)
     if args.impl == "reference":
         run_reference(args, cfg, rank)
     elif args.which == "backward":

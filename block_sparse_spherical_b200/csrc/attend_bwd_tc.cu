@@ -67,13 +67,17 @@ constexpr int TILE = BK * HD * 2;          // bytes of one 64x64 bf16 tile
 #define BSA_BWD_PIPES 2
 #endif
 constexpr int NPIPE = BSA_BWD_PIPES;       // independent pipelines per CTA (2 or 3)
-constexpr int NTHREADS = 32 * (2 * NPIPE + 4 * NPIPE);
+// setmaxnreg must be executed alike by the four warps of a warpgroup, so the control warps
+// (an MMA and a copy warp a pipeline) fill whole warpgroups: with three pipelines warps 6-7
+// only give their registers away.
+constexpr int kCtrlWarps = (2 * NPIPE + 3) / 4 * 4;
+constexpr int NTHREADS = 32 * (kCtrlWarps + 4 * NPIPE);
 // With three pipelines the unit tiles and the g·P / s·dS rows are single-buffered (64 KB of
 // shared memory a pipeline), and a register split gives the softmax threads their registers.
 constexpr int UB = NPIPE == 3 ? 1 : 2;     // unit tile buffers
 constexpr int DB = NPIPE == 3 ? 1 : 2;     // g·P / s·dS buffers
 constexpr int kCtrlRegs = 64, kSoftRegs = 112;
-constexpr int kRegsNeeded = 2 * NPIPE * 32 * kCtrlRegs + 4 * NPIPE * 32 * kSoftRegs;
+constexpr int kRegsNeeded = kCtrlWarps * 32 * kCtrlRegs + 4 * NPIPE * 32 * kSoftRegs;
 static_assert(NPIPE == 2 || kRegsNeeded <= 65536, "register split");
 constexpr uint32_t TMEM_COLS = 512;
 
@@ -543,17 +547,17 @@ attend_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_consta
     __syncthreads();
     fence_after();
     const uint32_t tmem = sh.tmem_base;
-    if (warp < 2 * NPIPE) {
+    if (warp < kCtrlWarps) {
         if constexpr (NPIPE == 3) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
         if (warp < NPIPE) {
             mma_role(p, sh.tiles[warp], sh.bars[warp], tmem, warp, abort_flag);
-        } else {
+        } else if (warp < 2 * NPIPE) {
             const int q = warp - NPIPE;
             loader_role(p, &tq, &tk, &tv, &to, sh.tiles[q], sh.bars[q], q, abort_flag);
         }
     } else {
         if constexpr (NPIPE == 3) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
-        const int q = (warp - 2 * NPIPE) >> 2;
+        const int q = (warp - kCtrlWarps) >> 2;
         softmax_role(p, sh.tiles[q], sh.bars[q], tmem, q, warp & 3, lane, abort_flag);
     }
     __syncwarp();
