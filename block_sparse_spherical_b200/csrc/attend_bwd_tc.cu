@@ -30,21 +30,29 @@
 //     atomic reductions over the full token range.
 // No atomics on dk, dv or dq: all three are bit-for-bit deterministic.
 //
-// Units are handed out round-robin to two independent pipelines per CTA
-// (persistent grid, one CTA per SM). Per pipeline:
-//   warp p (0-1)        : MMA warp (one elected lane issues)
-//   warp 2+p            : TMA copy warp: the unit's two tiles (key-major: K, V;
-//                         query-major: Q, dO; two buffers) and the step's two
-//                         (key-major: Q, dO; query-major: K, V; two stages)
-//   warps 4+4p..7+4p    : 128 softmax threads; thread (w, lane) owns row
+// Units are handed out round-robin to NPIPE independent pipelines per CTA
+// (persistent grid, one CTA per SM; three by default, two with -DBSA_BWD_PIPES=2).
+// Per pipeline p:
+//   warp p              : MMA warp (one elected lane issues)
+//   warp NPIPE+p        : TMA copy warp: the unit's two tiles (key-major: K, V;
+//                         query-major: Q, dO) and the step's two (key-major: Q,
+//                         dO; query-major: K, V; two stages)
+//   warps C+4p..C+3+4p  : 128 softmax threads; thread (w, lane) owns row
 //                         16(w%4) + lane%16 and columns 32(lane/16)..+31 of
 //                         the step's S and dP, and of the unit's accumulators
+// C = the control warps rounded up to whole warpgroups (4 for two pipelines, 8
+// for three, where warps 6-7 only give their registers away): setmaxnreg is
+// executed alike by the four warps of a warpgroup. With three pipelines the
+// control warps drop to 64 registers and the softmax warps rise to 112, and the
+// unit tiles and the g·P / s·dS rows are single-buffered (64 KB of shared
+// memory a pipeline); with two both are double-buffered and no split is needed.
 // Tensor memory (M=64 accumulators use 16 of the 32 lanes of each
 // sub-partition, so two share columns in the two lane halves):
 //   pipeline p: S  cols 128p..+63 lanes +0,  dP cols 128p..+63 lanes +16,
 //               dK (query-major: dQ) cols 128p+64..+63 lanes +0,
 //               dV cols 128p+64..+63 lanes +16
-//   per-step dQ of the compressed pass, pipeline p: cols 256..319, lanes +16p
+//   per-step dQ of the compressed pass, pipeline p: cols 128·NPIPE + 64(p/2)
+//               ..+63, lanes +16(p%2)
 // Every wait on an mbarrier is bounded (2 s); on expiry the kernel records a
 // timeout in the status word, the other roles stop at their next wait, the
 // copies and MMAs in flight are drained, TMEM is freed and the kernel returns.
@@ -64,7 +72,7 @@ constexpr int BK = 64;                     // rows of a tile
 constexpr int HD = 64;                     // head dim
 constexpr int TILE = BK * HD * 2;          // bytes of one 64x64 bf16 tile
 #ifndef BSA_BWD_PIPES
-#define BSA_BWD_PIPES 2
+#define BSA_BWD_PIPES 3
 #endif
 constexpr int NPIPE = BSA_BWD_PIPES;       // independent pipelines per CTA (2 or 3)
 // setmaxnreg must be executed alike by the four warps of a warpgroup, so the control warps

@@ -77,6 +77,9 @@ constexpr int NTHREADS = 32 * (2 * NSLOT + 4 * NSLOT);
 // exceed what the CTA was launched with; the host checks the compiled count.
 constexpr int kCtrlRegs = 48, kSoftRegs = 96;
 constexpr int kRegsNeeded = 2 * NSLOT * 32 * kCtrlRegs + 4 * NSLOT * 32 * kSoftRegs;
+// setmaxnreg must be executed alike by the four warps of a warpgroup: the 2·NSLOT control warps
+// have to fill whole warpgroups, or a mixed one could wait forever
+static_assert((2 * NSLOT) % 4 == 0, "control warps must fill whole warpgroups");
 constexpr uint32_t TMEM_COLS = 512;         // 128 columns per slot
 constexpr float kRescaleLog2 = 8.0f;        // lazy rescale threshold (factor 256)
 constexpr int kMaxMirrors = 7;              // output copies beyond `out` (8 ranks of one node)
@@ -108,7 +111,7 @@ static_assert(sizeof(SlotTiles) == (1 + 2 * NSTAGE) * TILE + (P_TMEM ? 1024 : 2 
 
 struct SlotBars {
     uint64_t q_full, q_empty;
-    uint64_t p_full[2], p_empty[2];
+    uint64_t p_full[2];
     uint64_t k_full[NSTAGE], k_empty[NSTAGE];
     uint64_t v_full[NSTAGE], v_empty[NSTAGE];
     uint64_t o_done[2];        // [step % 2]: P·V of that step complete
@@ -423,7 +426,6 @@ __device__ void mma_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint32_t 
                 }
                 commit(&B.o_done[pb]);
                 commit(&B.v_empty[vs]);
-                commit(&B.p_empty[pb]);
             }
             __syncwarp();
         }
@@ -582,10 +584,11 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 l_run *= alpha;
             }
             l_run += ls;
-            // ---- P (this thread's 32 columns of the row) -> shared memory buffer g%2,
-            //      K-major 128-byte swizzle, once P·V(g-2) has released that buffer
+            // ---- P (this thread's 32 columns of the row) -> buffer g%2. Its last reader,
+            //      P·V(g-2), was issued before S(g) by the same thread, and a commit tracks
+            //      every earlier MMA of its thread, so S(g) complete (waited above) means
+            //      P·V(g-2) has released the buffer: no wait of its own
             const int pb = g & 1;
-            if (!(ok = wait_all(&B.p_empty[pb], ((g >> 1) & 1) ^ 1))) break;
             if (P_TMEM) {
                 // P (bf16 pairs) into this row's lanes of P buffer pb: the A operand of P·V
                 tmem_st16_pairs(tP + 32u * pb, pk);
@@ -661,7 +664,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
             mbar_init(&B.q_empty, 1);
             for (int b = 0; b < 2; ++b) {
                 mbar_init(&B.p_full[b], 128);
-                mbar_init(&B.p_empty[b], 1);
             }
             for (int b = 0; b < NSTAGE; ++b) {
                 mbar_init(&B.k_full[b], 1);

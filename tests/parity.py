@@ -76,15 +76,18 @@ def to_np(t: torch.Tensor) -> np.ndarray:
     return t.cpu().numpy()
 
 
-def check_slab(cfg, slab: int, gpu: dict, max_rows: int | None):
+def check_slab(cfg, slab: int, gpu: dict, max_rows: int | None, q_scale: float = 1.0):
     """Compare one slab's GPU results with the oracle on sampled query blocks.
 
     gpu holds numpy arrays for this slab: qbar/kbar/vbar [m,d], o_cg [m,d],
-    idx [m,n], out [N,d] (any may be missing). Returns a summary dict.
+    idx [m,n], out [N,d] (any may be missing). q_scale multiplies the seeded q
+    (a power of two, so that the GPU's bf16 q scaled the same way is exact).
+    Returns a summary dict.
     """
     s = make_slab(cfg, slab)
     bk, n, w = cfg.block_size, cfg.top_n, cfg.window_blocks
     q, k, v, g = (x.astype(np.float64) for x in (s.q, s.k, s.v, s.gates))
+    q = q * q_scale
     qb, kb, vb = (oracle.pool(x, bk) for x in (q, k, v))
     summary = {"near_ties": 0, "out_max": 0.0, "out_mean": 0.0}
     for name, ob in (("qbar", qb), ("kbar", kb), ("vbar", vb)):
