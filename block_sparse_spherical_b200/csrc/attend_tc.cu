@@ -236,6 +236,14 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                        __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
+// 16 consecutive values x[e]·f as bf16 at dst (32 B, 16-byte aligned).
+__device__ __forceinline__ void store_row16(__nv_bfloat16 *dst, const float *x, float f) {
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+        d4[c] = make_uint4(pack_bf16(x[8 * c] * f, x[8 * c + 1] * f), pack_bf16(x[8 * c + 2] * f, x[8 * c + 3] * f),
+                           pack_bf16(x[8 * c + 4] * f, x[8 * c + 5] * f), pack_bf16(x[8 * c + 6] * f, x[8 * c + 7] * f));
+}
 // 32 consecutive values x[e]·f as bf16 at dst (64 B, 16-byte aligned).
 __device__ __forceinline__ void store_row32(__nv_bfloat16 *dst, const float *x, float f) {
     uint4 *d4 = reinterpret_cast<uint4 *>(dst);
@@ -526,15 +534,21 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             uint32_t pk[16];
             float ls = 0.f;
             if (valid) {
-                // p = 2^(s·scale·log2e − m), two columns per packed FMA, two independent sums
+                // p = 2^(s·scale·log2e − m), two columns per packed FMA. In three phases (all
+                // exponents, then all exponentials, then packing and the sums), so that the
+                // warp's in-order issue never waits on one exp-unit result while later
+                // independent exponentials could still be queued
                 const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_used, -m_used);
+                float2 x[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) x[c] = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) x[c] = (c < POLY_PAIRS) ? exp2_poly2(x[c]) : make_float2(ex2(x[c].x), ex2(x[c].y));
                 float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
-                    const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
-                    const float2 e = (c < POLY_PAIRS) ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
-                    pk[c] = pack_bf16(e.x, e.y);
-                    acc2[c & 1] = __fadd2_rn(acc2[c & 1], e);
+                    pk[c] = pack_bf16(x[c].x, x[c].y);
+                    acc2[c & 1] = __fadd2_rn(acc2[c & 1], x[c]);
                 }
                 const float2 t2 = __fadd2_rn(acc2[0], acc2[1]);
                 ls = t2.x + t2.y;
@@ -554,19 +568,27 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
                 // this row's lanes of the other lane half until the epilogue
                 const float l = l_sel + __shfl_xor_sync(FULL, l_sel, 16);
                 const float inv = l > 0.f ? g_fg / l : 0.f;
-                float a[32];
-                tmem_ld16(tO, a);
-                tmem_ld16(tO + 16, a + 16);
-                tmem_wait_ld();
-                if constexpr (MODE == 1) {     // training: o_FG and its row log-sum-exp
-                    const float inv1 = l > 0.f ? 1.f / l : 0.f;
-                    store_row32(p.o_fg + tok * HD + 32 * ch, a, inv1);
+                if constexpr (MODE == 1)       // training: the row log-sum-exp of o_FG
                     if (ch == 0) p.lse[tok * 2] = (m_sel + __log2f(l)) * 0.69314718055994531f;
-                }
 #pragma unroll
-                for (int e = 0; e < 32; ++e) a[e] = fmaf(g_cg, __ldg(ocg + e), a[e] * inv);
-                tmem_st16(tA, a);
-                tmem_st16(tA + 16, a + 16);
+                for (int hh = 0; hh < 2; ++hh) {   // 16 columns at a time (register pressure)
+                    float a[16];
+                    tmem_ld16(tO + 16 * hh, a);
+                    tmem_wait_ld();
+                    if constexpr (MODE == 1) {     // training: o_FG itself
+                        const float inv1 = l > 0.f ? 1.f / l : 0.f;
+                        store_row16(p.o_fg + tok * HD + 32 * ch + 16 * hh, a, inv1);
+                    }
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {   // o_cg: one 256-byte row per query block
+                        const float4 c4 = __ldg(reinterpret_cast<const float4 *>(ocg) + 4 * hh + e4);
+                        a[4 * e4] = fmaf(g_cg, c4.x, a[4 * e4] * inv);
+                        a[4 * e4 + 1] = fmaf(g_cg, c4.y, a[4 * e4 + 1] * inv);
+                        a[4 * e4 + 2] = fmaf(g_cg, c4.z, a[4 * e4 + 2] * inv);
+                        a[4 * e4 + 3] = fmaf(g_cg, c4.w, a[4 * e4 + 3] * inv);
+                    }
+                    tmem_st16(tA + 16 * hh, a);
+                }
                 tmem_wait_st();
             } else if (touch_o) {
                 // rows whose running max grew by more than 2^8: rescale their O and sum
