@@ -24,10 +24,13 @@
 //                into tf32 parts and store them in the MMA's 128-byte-swizzled
 //                K-major layout (V transposed: rows are features, keys run
 //                along K); K runs one tile ahead of V
-//   warp 8     : tensor-core warp (one elected lane issues): S(j) = Q·K(j)ᵀ
-//                into TMEM buffer j%2, then O(j-1) = P(j-1)·V(j-1) into TMEM
-//                buffer (j-1)%2
-//   warps 9-11 : complete the third warpgroup (registers are allocated by
+//   warp 8     : S warp (one elected lane issues): S(j) = Q·K(j)ᵀ into TMEM
+//                buffer j%2
+//   warp 9     : P·V warp (one elected lane issues): O(j) = P(j)·V(j) into
+//                TMEM buffer j%2. Two issuing threads: one thread issues a
+//                tcgen05.mma about every 55-60 cycles at best, and a tile
+//                needs 48 of them
+//   warps 10-11: complete the third warpgroup (registers are allocated by
 //                whole warpgroups) and only give their registers away
 // The row threads hold the tile's logits, their output row and their top-n
 // list in registers; a register split (setmaxnreg) moves registers to them
@@ -74,7 +77,7 @@ struct alignas(1024) Smem {
     uint8_t vhi[2][KROWS], vlo[2][KROWS];           // B of P·V, [region]: feature x key; region c: keys 32c..
     uint8_t phi[2][RROWS], plo[2][RROWS];           // A of P·V, [region]: row x key
     uint64_t q_full, k_full[2], k_empty[2], v_full, v_empty;
-    uint64_t s_full[2], s_free[2], p_full, p_empty, o_full[2], o_free[2], drain;
+    uint64_t s_full[2], s_free[2], p_full, p_empty, o_full[2], o_free[2], drain, drain_pv;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -106,10 +109,13 @@ __device__ __forceinline__ void store_split(uint8_t *hi, uint8_t *lo, uint32_t o
     h.y = tf32_hi(x.y);
     h.z = tf32_hi(x.z);
     h.w = tf32_hi(x.w);
-    l.x = x.x - h.x;
-    l.y = x.y - h.y;
-    l.z = x.z - h.z;
-    l.w = x.w - h.w;
+    // x - h, exact, two lanes per packed FMA
+    const float2 l01 = __ffma2_rn(make_float2(h.x, h.y), make_float2(-1.f, -1.f), make_float2(x.x, x.y));
+    const float2 l23 = __ffma2_rn(make_float2(h.z, h.w), make_float2(-1.f, -1.f), make_float2(x.z, x.w));
+    l.x = l01.x;
+    l.y = l01.y;
+    l.z = l23.x;
+    l.w = l23.y;
     *reinterpret_cast<float4 *>(hi + off) = h;
     *reinterpret_cast<float4 *>(lo + off) = l;
 }
@@ -260,25 +266,11 @@ __device__ __forceinline__ void mma_3pass(uint32_t d, const uint8_t *ah0, const 
         mma_tf32(d, al[kk >> 2] + 2 * (kk & 3), bh[kk >> 2] + 2 * (kk & 3), kIdesc, 1u);
 }
 
-__device__ void mma_role(const Args &a, Smem &sh, uint32_t tmem, int T, volatile int *abort_flag) {
+// S(j) = Q·K(j)ᵀ into TMEM buffer j%2, for every key tile j.
+__device__ void mma_s_role(const Args &a, Smem &sh, uint32_t tmem, int T, volatile int *abort_flag) {
     const bool leader = elect_one();
     auto wait_w = [&](uint64_t *b, uint32_t par) -> bool {
         return __all_sync(0xffffffffu, mbar_try_wait(b, par) || wait_bar(b, par, abort_flag, a.status));
-    };
-    auto issue_pv = [&](int i) -> bool {   // O(i%2) = P(i)·V(i)
-        if (!wait_w(&sh.p_full, i & 1) || !wait_w(&sh.v_full, i & 1) ||
-            !wait_w(&sh.o_free[i & 1], ((i >> 1) & 1) ^ 1))
-            return false;
-        fence_after();
-        if (leader) {
-            mma_3pass(tmem + 128 + 64 * (i & 1), sh.phi[0], sh.phi[1], sh.plo[0], sh.plo[1], sh.vhi[0], sh.vhi[1],
-                      sh.vlo[0], sh.vlo[1]);
-            commit(&sh.o_full[i & 1]);
-            commit(&sh.v_empty);
-            commit(&sh.p_empty);
-        }
-        __syncwarp();
-        return true;
     };
     bool ok = wait_w(&sh.q_full, 0);
     for (int j = 0; ok && j < T; ++j) {
@@ -293,15 +285,38 @@ __device__ void mma_role(const Args &a, Smem &sh, uint32_t tmem, int T, volatile
             commit(&sh.k_empty[st]);
         }
         __syncwarp();
-        if (j > 0 && !(ok = issue_pv(j - 1))) break;
     }
-    if (ok && T > 0) ok = issue_pv(T - 1);
     // every MMA this thread issued must be complete before TMEM is freed
     if (leader) commit(&sh.drain);
     __syncwarp();
     drain_bar(&sh.drain, 0);
 }
 
+// O(i) = P(i)·V(i) into TMEM buffer i%2, for every key tile i.
+__device__ void mma_pv_role(const Args &a, Smem &sh, uint32_t tmem, int T, volatile int *abort_flag) {
+    const bool leader = elect_one();
+    auto wait_w = [&](uint64_t *b, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, mbar_try_wait(b, par) || wait_bar(b, par, abort_flag, a.status));
+    };
+    bool ok = true;
+    for (int i = 0; ok && i < T; ++i) {
+        if (!(ok = wait_w(&sh.p_full, i & 1) && wait_w(&sh.v_full, i & 1) &&
+                   wait_w(&sh.o_free[i & 1], ((i >> 1) & 1) ^ 1)))
+            break;
+        fence_after();
+        if (leader) {
+            mma_3pass(tmem + 128 + 64 * (i & 1), sh.phi[0], sh.phi[1], sh.plo[0], sh.plo[1], sh.vhi[0], sh.vhi[1],
+                      sh.vlo[0], sh.vlo[1]);
+            commit(&sh.o_full[i & 1]);
+            commit(&sh.v_empty);
+            commit(&sh.p_empty);
+        }
+        __syncwarp();
+    }
+    if (leader) commit(&sh.drain_pv);
+    __syncwarp();
+    drain_bar(&sh.drain_pv, 0);
+}
 
 // lv/li = the first NSEL entries of s (keys 0..NSEL-1) sorted by (value
 // descending, key ascending): a bitonic network on registers.
@@ -387,7 +402,12 @@ __device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter
         const float m_i = (i & 1) ? m_odd : m_even;
         const float f = ex2(m_acc - m_i);
 #pragma unroll
-        for (int c = 0; c < D; ++c) o[c] = fmaf(o[c], f, part[c]);
+        for (int c = 0; c < D / 2; ++c) {
+            const float2 r2 = __ffma2_rn(make_float2(o[2 * c], o[2 * c + 1]), make_float2(f, f),
+                                         make_float2(part[2 * c], part[2 * c + 1]));
+            o[2 * c] = r2.x;
+            o[2 * c + 1] = r2.y;
+        }
         m_acc = m_i;
         return true;
     };
@@ -442,11 +462,25 @@ __device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter
         // ---- online softmax (log2 domain) of the row
         const float mt = fmax3(fmax3(gm[0], gm[1], gm[2]), fmax3(gm[3], gm[4], gm[5]), fmaxf(gm[6], gm[7]));
         const float m_new = fmaxf(m_run, mt * a.sl2);
-        float ls = 0.f;
+        // exponents, then all exponentials, then four packed partial sums: in-order issue
+        // never waits on one exp-unit result while later independent ones could be queued
+        float ls;
+        {
+            const float2 sc2 = make_float2(a.sl2, a.sl2), nm2 = make_float2(-m_new, -m_new);
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-            s[c] = ex2(fmaf(s[c], a.sl2, -m_new));
-            ls += s[c];
+            for (int c = 0; c < BN / 2; ++c) {
+                const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
+                s[2 * c] = x.x;
+                s[2 * c + 1] = x.y;
+            }
+#pragma unroll
+            for (int c = 0; c < BN; ++c) s[c] = ex2(s[c]);
+            float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                              make_float2(0.f, 0.f)};
+#pragma unroll
+            for (int c = 0; c < BN / 2; ++c) acc4[c & 3] = __fadd2_rn(acc4[c & 3], make_float2(s[2 * c], s[2 * c + 1]));
+            const float2 t2 = __fadd2_rn(__fadd2_rn(acc4[0], acc4[1]), __fadd2_rn(acc4[2], acc4[3]));
+            ls = t2.x + t2.y;
         }
         l_run = fmaf(l_run, ex2(m_run - m_new), ls);
         m_run = m_new;
@@ -524,6 +558,7 @@ compress_tc_kernel(const float *__restrict__ qbar, const float *__restrict__ kba
         mbar_init(&sh.p_full, 128);
         mbar_init(&sh.p_empty, 1);
         mbar_init(&sh.drain, 1);
+        mbar_init(&sh.drain_pv, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sh.k_full[b], kFill);
             mbar_init(&sh.k_empty[b], 1);
@@ -557,7 +592,9 @@ compress_tc_kernel(const float *__restrict__ qbar, const float *__restrict__ kba
             convert_role(a, sh, threadIdx.x - 128, row0, T, abort_flag);
         }
         if (warp == 8)
-            mma_role(a, sh, tmem, T, abort_flag);
+            mma_s_role(a, sh, tmem, T, abort_flag);
+        else if (warp == 9)
+            mma_pv_role(a, sh, tmem, T, abort_flag);
     }
     __syncwarp();
 
