@@ -23,7 +23,7 @@ EXPORTS = ("bsa_pool", "bsa_compress_select", "bsa_compress_select_ws", "bsa_fin
            "bsa_workspace_size", "bsa_forward", "bsa_check_status", "bsa_status_string", "bsa_forward_noalloc",
            "bsa_forward_train", "bsa_backward_workspace_size", "bsa_backward", "bsa_permute_tokens",
            "bsa_latlon_healpix_plan", "bsa_latlon_workspace_size", "bsa_latlon_to_healpix", "bsa_forward_mirrored")
-TESTING_EXPORTS = ("bsa_testing_fine_attention_withhold", "bsa_testing_exp2")
+TESTING_EXPORTS = ("bsa_testing_fine_attention_withhold", "bsa_testing_exp2", "bsa_testing_mma_rate")
 
 
 class BsaConfig(ctypes.Structure):
@@ -71,6 +71,7 @@ def load() -> ctypes.CDLL:
                                   ctypes.c_float, P, P, P, P, P, P, P, S, P, P],
         "bsa_testing_fine_attention_withhold": [C, P, P, P, P, P, P, P, P, ctypes.c_int64, P],
         "bsa_testing_exp2": [P, P, ctypes.c_int64, ctypes.c_int32, P],
+        "bsa_testing_mma_rate": [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, P, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -204,6 +205,11 @@ def bsa_forward_mirrored(cfg: BsaConfig, q, k, v, gates, out, mirrors, sel_idx_o
     _check("bsa_forward_mirrored", load().bsa_forward_mirrored(
         ctypes.byref(cfg), _ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(out), arr, len(mirrors),
         _ptr(sel_idx_out), _ptr(workspace), workspace_bytes, _stream(stream)))
+
+
+def bsa_testing_mma_rate(m: int, n: int, warps: int, cycles, stream=None) -> None:
+    """Test hook: each of `warps` warps' cycles for 256 back-to-back m x n bf16 tcgen05.mma (K=16)."""
+    _check("bsa_testing_mma_rate", load().bsa_testing_mma_rate(m, n, warps, _ptr(cycles), _stream(stream)))
 
 
 def bsa_check_status(status_word, stream=None) -> int:

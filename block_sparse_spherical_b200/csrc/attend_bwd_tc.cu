@@ -444,15 +444,30 @@ __device__ void softmax_role(const BwdParams &p, PipeTiles &S, PipeBars &B, uint
             // of a selected block outside [0, m)
             const int kvalid = p.dense ? min(32, max(0, p.valid - (x.T * BK + 32 * ch))) : (stp.valid ? 32 : 0);
             uint32_t ppk[16], dpk[16];
+            // exponents, then all exponentials, then the products: in-order issue never waits
+            // on one exp-unit result while later independent ones could be queued
+            {
+                const float2 sc2 = make_float2(sl2, sl2), nl2 = make_float2(-lse2, -lse2);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                float p0 = ex2(fmaf(sv[2 * e], sl2, -lse2)), p1 = ex2(fmaf(sv[2 * e + 1], sl2, -lse2));
-                if (2 * e >= kvalid) p0 = 0.f;
-                if (2 * e + 1 >= kvalid) p1 = 0.f;
-                const float d0 = sc * p0 * fmaf(gate, dp[2 * e], -D);
-                const float d1 = sc * p1 * fmaf(gate, dp[2 * e + 1], -D);
-                ppk[e] = pack_bf16x2(gate * p0, gate * p1);
-                dpk[e] = pack_bf16x2(d0, d1);
+                for (int e = 0; e < 16; ++e) {
+                    const float2 x = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), sc2, nl2);
+                    sv[2 * e] = x.x;
+                    sv[2 * e + 1] = x.y;
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sv[e] = ex2(sv[e]);
+            {
+                const float2 g2 = make_float2(gate, gate), nd2 = make_float2(-D, -D), s2 = make_float2(sc, sc);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float2 p2 = make_float2(2 * e < kvalid ? sv[2 * e] : 0.f, 2 * e + 1 < kvalid ? sv[2 * e + 1] : 0.f);
+                    const float2 t2 = __ffma2_rn(g2, make_float2(dp[2 * e], dp[2 * e + 1]), nd2);   // g·dP − D
+                    const float2 d2 = __fmul2_rn(__fmul2_rn(s2, p2), t2);                          // s·P·(g·dP − D)
+                    const float2 gp = __fmul2_rn(g2, p2);
+                    ppk[e] = pack_bf16x2(gp.x, gp.y);
+                    dpk[e] = pack_bf16x2(d2.x, d2.y);
+                }
             }
             // ---- s·dS (and g·P) rows into buffer g%2 once the MMAs of step g-2 released it
             const int b = g % DB;

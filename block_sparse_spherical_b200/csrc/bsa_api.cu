@@ -611,3 +611,13 @@ extern "C" bsa_status bsa_testing_exp2(const float *x, float *y, int64_t n, int3
     if (n == 0) return BSA_OK;
     return from_cuda(bsa::launch_exp2_eval(x, y, n, poly, stream));
 }
+
+// Test hook (include/bsa_testing.h): tcgen05.mma issue and execution rate of an m x n tile.
+extern "C" bsa_status bsa_testing_mma_rate(int32_t m, int32_t n, int32_t warps, int64_t *cycles,
+                                           cudaStream_t stream) {
+    if (!cycles || (m != 64 && m != 128) || (n != 64 && n != 128 && n != 256) ||
+        (warps != 1 && warps != 2 && warps != 4))
+        return BSA_ERR_INVALID_ARG;
+    if ((uintptr_t)cycles & 7u) return BSA_ERR_ALIGNMENT;
+    return from_cuda(bsa::launch_mma_rate(m, n, warps, reinterpret_cast<long long *>(cycles), stream));
+}

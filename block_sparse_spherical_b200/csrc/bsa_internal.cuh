@@ -72,6 +72,10 @@ cudaError_t launch_interp(int64_t batch, int64_t n_tgt, int64_t n_src, int64_t d
 
 // Test hook: the fine-attention kernel's exp2 on the FMA pipe (poly != 0) or the exp unit.
 cudaError_t launch_exp2_eval(const float *x, float *y, int64_t n, int poly, cudaStream_t stream);
+// Test hook: cycles of `warps` threads (one per warp) each issuing 256 back-to-back bf16 tcgen05.mma
+// of an m x n tile (K = 16) through completion, into cycles[0..warps) (device); -1 on a timeout.
+cudaError_t launch_mma_rate(int m, int n, int warps, long long *cycles, cudaStream_t stream);
+int mma_rate_mmas_per_warp();
 
 // ---- backward (training) ------------------------------------------------
 

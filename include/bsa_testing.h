@@ -35,6 +35,20 @@ BSA_API bsa_status bsa_testing_fine_attention_withhold(const bsa_config *cfg, co
  */
 BSA_API bsa_status bsa_testing_exp2(const float *x, float *y, int64_t n, int32_t poly, cudaStream_t stream);
 
+/*
+ * Tensor-pipe rate microbenchmark: one CTA, `warps` (1, 2 or 4) warps each with
+ * one thread issuing 256 back-to-back tcgen05.mma (kind::f16, bf16 zero
+ * operands in shared memory, K = 16) of an m x n tile (m 64 or 128, n 64, 128
+ * or 256) into its own tensor-memory columns, then waiting (bounded) for them.
+ * cycles (device, 8-byte aligned, `warps` entries) receives each warp's clock
+ * cycles from its first issue to completion, or -1 if the wait expired. The
+ * multiply-add rate of the SM is m*n*16*256*warps / max(cycles). Used to
+ * measure the M = 64 ceiling of the fine-attention kernel (an M = 64 tile
+ * drives half of the tensor datapath). Returns BSA_ERR_INVALID_ARG for other
+ * shapes or warp counts.
+ */
+BSA_API bsa_status bsa_testing_mma_rate(int32_t m, int32_t n, int32_t warps, int64_t *cycles, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
