@@ -1,28 +1,24 @@
 // Selection branch (b), local branch (c) and the gated combine of the BSA
-// section (MOSAIC note) on the sm_100a tensor cores: bf16 inputs, block 64,
-// head_dim 64, fp32 accumulation in tensor memory.
+// section (MOSAIC note) on the sm_100a tensor cores: bf16 inputs, blocks of
+// 64·R tokens (R = 1, 4 or 16), head_dim 64, fp32 accumulation in tensor memory.
 //
-// Thanks to the NESTED order every key/value block is one contiguous 8 KB
-// span, so each is a single TMA box (64 rows x 128 B, 128-byte swizzle)
-// copied straight into the layout tcgen05.mma reads. Per query block the
-// kernel streams its n selected blocks and then its 2w+1 local blocks; for
-// each block it runs S = Q·Kᵀ (tcgen05.mma, M=64 N=64 K=64) into TMEM, an
-// online softmax on the CUDA cores, and O += P·V (tcgen05.mma, P from shared
-// memory). The selection branch's output is folded, together with the
-// compressed branch, into a per-thread accumulator (acc = g_CG·o_CG +
-// g_FG·o_FG) before the local branch reuses the same TMEM accumulator; the
-// epilogue adds g_L·o_L and stores bf16. acc is held as fp16 pairs under a
-// power-of-two scale per thread that puts its largest entry in [2^14, 2^15)
-// (relative rounding 2^-11, eight times finer than the bf16 output's): in
-// fp32 it would not fit the softmax warps' register budget and would spill.
+// Thanks to the NESTED order every key/value tile of 64 rows is one contiguous
+// 8 KB span, so each is a single TMA box (64 rows x 128 B, 128-byte swizzle)
+// copied straight into the layout tcgen05.mma reads. Per 64-row query tile the
+// kernel streams the tiles of its block's n selected blocks and then of its
+// 2w+1 local blocks; for each key tile it runs S = Q·Kᵀ (tcgen05.mma, M=64
+// N=64 K=64) into TMEM, an online softmax on the CUDA cores (lazy rescaling),
+// and O += P·V (tcgen05.mma with P, bf16, read from TMEM). When the selection
+// branch ends, its output is folded with the compressed branch into acc =
+// g_CG·o_CG + g_FG·o_FG, held in fp32 in TMEM (the other lane half), and the
+// local branch starts a fresh O; the epilogue adds g_L·o_L and stores bf16.
 //
 // Organisation: a persistent grid of one CTA per SM, 768 threads, four
-// independent pipelines ("slots") per CTA, each working on one query block at
-// a time. A slot's M=64 accumulators (S, then O) live in TMEM lanes 0-15 of
-// each 32-lane sub-partition, in its own 128-column range. Four slots give
-// four concurrent MMA issue streams (a single stream of M=64 N=64 MMAs
-// cannot keep the tensor pipe busy) and let the pipelines drift out of phase
-// so that their softmax phases do not all contend for the exp unit at once.
+// independent pipelines ("slots") per CTA, each working on one query tile at a
+// time in its own 128 TMEM columns. Four slots give four concurrent MMA issue
+// streams (one thread issues a 64x64 tcgen05.mma about every 55 cycles, half
+// of what the tensor pipe takes) and let the pipelines drift out of phase so
+// that their softmax phases do not all contend for the exp unit at once.
 //   warp s (0-3)       : MMA warp of slot s
 //   warp 4+s           : TMA copy warp of slot s: Q, then K one step ahead of V
 //   warps 8+4s..11+4s  : softmax + epilogue warpgroup of slot s; with the
@@ -180,6 +176,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *r) {
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 32;"
         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
           "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+        : "r"(taddr));
+}
+// 16 lanes x 32 columns twice: thread t < 16 reads lane (base + t) columns [col, col+32),
+// thread t >= 16 lane (base + t - 16) columns [col+32, col+64): one row half per thread.
+__device__ __forceinline__ void tmem_ld_row32(uint32_t taddr, float *r) {
+    uint32_t *u = reinterpret_cast<uint32_t *>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15]),
+          "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]),
+          "=r"(u[24]), "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
         : "r"(taddr));
 }
 // 16 lanes x 16 columns: thread t < 16 writes lane (base + t) columns [col, col+16), thread
@@ -520,8 +530,7 @@ __device__ void softmax_role(const TcParams &p, SlotTiles &S, SlotBars &B, uint3
             if (!(ok = wait_all(&B.s_full, g & 1))) break;
             fence_after();
             float s[32];
-            tmem_ld16(tS, s);
-            tmem_ld16(tS + 16, s + 16);
+            tmem_ld_row32(tS, s);
             tmem_wait_ld();
             fence_before();
             mbar_arrive(&B.s_free);            // every softmax thread arrives (count 128)

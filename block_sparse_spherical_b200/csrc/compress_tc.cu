@@ -16,25 +16,28 @@
 //
 // One CTA owns 128 query blocks (rows) of one slab and streams the slab's key
 // blocks in tiles of 64 (the m×m logit matrix never leaves the SM):
-//   warps 0-3  : one thread per row (TMEM lane): reads the row's 64 logits of
-//                the tile, updates its sorted top-n list and the online
-//                softmax, stores the row's P in tf32 parts for the P·V MMA and
-//                folds the previous tile's O into its fp32 accumulator
-//   warps 4-7  : converters: read q̄, k̄, v̄ rows (fp32, L2-resident), split them
+//   warps 0-7  : two threads per row (TMEM lane): thread (q = warp%4, h = warp/4)
+//                owns row 32q + lane and the keys 32h..32h+31 of each tile. It
+//                reads those 32 logits, updates its own sorted top-n list and
+//                online softmax, stores its half of P in tf32 parts for the
+//                P·V MMA and folds its half's previous P·V into an fp32
+//                accumulator. At the end half 1 hands its state to half 0
+//                through tensor memory and half 0 merges both.
+//   warps 8-11 : converters: read q̄, k̄, v̄ rows (fp32, L2-resident), split them
 //                into tf32 parts and store them in the MMA's 128-byte-swizzled
 //                K-major layout (V transposed: rows are features, keys run
 //                along K); K runs one tile ahead of V
-//   warp 8     : S warp (one elected lane issues): S(j) = Q·K(j)ᵀ into TMEM
+//   warp 12    : S warp (one elected lane issues): S(j) = Q·K(j)ᵀ into TMEM
 //                buffer j%2
-//   warp 9     : P·V warp (one elected lane issues): O(j) = P(j)·V(j) into
-//                TMEM buffer j%2. Two issuing threads: one thread issues a
-//                tcgen05.mma about every 55-60 cycles at best, and a tile
-//                needs 48 of them
-//   warps 10-11: complete the third warpgroup (registers are allocated by
+//   warp 13    : P·V warp (one elected lane issues): O_h(j) = P(j)[:, half h] ·
+//                V(j)[half h, :] into TMEM buffer j%2, both halves. Two issuing
+//                threads: one thread issues a tcgen05.mma about every 55-60
+//                cycles at best, and a tile needs 48 of them
+//   warps 14-15: complete the fourth warpgroup (registers are allocated by
 //                whole warpgroups) and only give their registers away
-// The row threads hold the tile's logits, their output row and their top-n
-// list in registers; a register split (setmaxnreg) moves registers to them
-// from the other warps, by whole warpgroups.
+// The row threads hold their logits, output row and top-n list in registers;
+// a register split (setmaxnreg) moves registers to them from the other warps,
+// by whole warpgroups.
 // Given a workspace, a split kernel first writes every tile's tf32 parts, as
 // the byte image of its shared-memory layout, once per slab; the converter
 // warps then give way to one copy thread (bulk copies of those images), and no
@@ -55,17 +58,17 @@ using namespace tc;
 constexpr int BM = 128;                    // query blocks per CTA
 constexpr int BN = 64;                     // key blocks per tile
 constexpr int D = 64;                      // head dim
-constexpr int NTHREADS = 32 * 12;          // three whole warpgroups (see the register split)
+constexpr int NTHREADS = 32 * 16;          // four whole warpgroups (see the register split)
 constexpr int RROWS = 128 * 128;           // bytes of one 128-row swizzled region
 constexpr int KROWS = 64 * 128;            // bytes of one 64-row swizzled region
-constexpr uint32_t TMEM_COLS = 256;        // S buffers at columns 0 and 64, O buffers at 128 and 192
-// Register split: the CTA is launched with 168 registers a thread (384
-// threads, one CTA per SM); the row warpgroup rises to kRowRegs, the other
-// two warpgroups drop to kCtlRegs. 128·kRowRegs + 256·kCtlRegs must not exceed
-// 384·168 (the host checks the compiled launch count), or setmaxnreg.inc would
+constexpr uint32_t TMEM_COLS = 512;        // S buffers at 0 and 64; O(buffer b, half h) at 128 + 128b + 64h
+// Register split: the CTA is launched with 128 registers a thread (512
+// threads, one CTA per SM); the two row warpgroups rise to kRowRegs, the other
+// two warpgroups drop to kCtlRegs. 256·kRowRegs + 256·kCtlRegs must not exceed
+// 512·128 (the host checks the compiled launch count), or setmaxnreg.inc would
 // wait forever.
-constexpr int kRowRegs = 240, kCtlRegs = 128;
-constexpr int kRegsNeeded = 128 * kRowRegs + 256 * kCtlRegs;
+constexpr int kRowRegs = 184, kCtlRegs = 72;
+constexpr int kRegsNeeded = 256 * kRowRegs + 256 * kCtlRegs;
 
 // instruction descriptor: D f32, A and B tf32, both K-major, M = 128, N = 64
 constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(64 >> 3) << 17) |
@@ -78,6 +81,7 @@ struct alignas(1024) Smem {
     uint8_t phi[2][RROWS], plo[2][RROWS];           // A of P·V, [region]: row x key
     uint64_t q_full, k_full[2], k_empty[2], v_full, v_empty;
     uint64_t s_full[2], s_free[2], p_full, p_empty, o_full[2], o_free[2], drain, drain_pv;
+    uint64_t merge[4];                              // [row quarter]: half 1's final state handed over
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -267,6 +271,19 @@ __device__ __forceinline__ void mma_3pass(uint32_t d, const uint8_t *ah0, const 
 }
 
 // S(j) = Q·K(j)ᵀ into TMEM buffer j%2, for every key tile j.
+// D = A·Bᵀ in three tf32 passes over K = 32 (one 128-byte region of each operand): 12 MMAs.
+__device__ __forceinline__ void mma_3pass_k32(uint32_t d, const uint8_t *ah0, const uint8_t *al0, const uint8_t *bh0,
+                                              const uint8_t *bl0) {
+    const uint64_t ah = desc_kmajor_sw128(ah0), al = desc_kmajor_sw128(al0);
+    const uint64_t bh = desc_kmajor_sw128(bh0), bl = desc_kmajor_sw128(bl0);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) mma_tf32(d, ah + 2 * kk, bh + 2 * kk, kIdesc, kk > 0);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) mma_tf32(d, ah + 2 * kk, bl + 2 * kk, kIdesc, 1u);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) mma_tf32(d, al + 2 * kk, bh + 2 * kk, kIdesc, 1u);
+}
+
 __device__ void mma_s_role(const Args &a, Smem &sh, uint32_t tmem, int T, volatile int *abort_flag) {
     const bool leader = elect_one();
     auto wait_w = [&](uint64_t *b, uint32_t par) -> bool {
@@ -305,8 +322,10 @@ __device__ void mma_pv_role(const Args &a, Smem &sh, uint32_t tmem, int T, volat
             break;
         fence_after();
         if (leader) {
-            mma_3pass(tmem + 128 + 64 * (i & 1), sh.phi[0], sh.phi[1], sh.plo[0], sh.plo[1], sh.vhi[0], sh.vhi[1],
-                      sh.vlo[0], sh.vlo[1]);
+            // O_h(i) = P(i)[:, keys of half h] · V(i)[keys of half h, :]: K = 32 from region h
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+                mma_3pass_k32(tmem + 128 + 128 * (i & 1) + 64 * hh, sh.phi[hh], sh.plo[hh], sh.vhi[hh], sh.vlo[hh]);
             commit(&sh.o_full[i & 1]);
             commit(&sh.v_empty);
             commit(&sh.p_empty);
@@ -368,12 +387,42 @@ __device__ __forceinline__ void list_insert(float *lv, int *li, float v, int j) 
     }
 }
 
+// 32 lanes x 16 columns: thread t of the warp reads / writes TMEM lane (base + t), columns [col, col+16).
+__device__ __forceinline__ void tmem_ld16c(uint32_t taddr, float *r) {
+    uint32_t *u = reinterpret_cast<uint32_t *>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16c(uint32_t taddr, const float *r) {
+    const uint32_t *u = reinterpret_cast<const uint32_t *>(r);
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "r"(u[8]),
+        "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
+        : "memory");
+}
+
+// (v, i) ranks before (w, k) in the selection order (logit descending, block index ascending)
+__device__ __forceinline__ bool ranks_before(float v, int i, float w, int k) { return v > w || (v == w && i < k); }
+
+// Row threads: two per row. Thread (q, h, lane) owns row r = 32q + lane (TMEM lane) and, of
+// every key tile, the 32 keys 32h..32h+31: their logits, its own sorted top-n list of those keys,
+// its own online softmax (running max and sum) and its own P·V accumulator O_h over them. The
+// two halves never exchange anything per tile; at the end half 1 hands its state to half 0
+// through tensor memory and half 0 merges: the lists by the selection order, the softmax states
+// by rescaling both to the larger maximum.
 template <int NSEL>
-__device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter, int lane, int row0, int T,
-                             volatile int *abort_flag) {
-    const int r = 32 * quarter + lane;     // row of the tile = TMEM lane
+__device__ void row_role(const Args &a, Smem &sh, uint32_t tmem, int q, int h, int lane, int row0, int T,
+                         volatile int *abort_flag) {
+    const int r = 32 * q + lane;           // row of the tile = TMEM lane
     const int row = row0 + r;
-    const uint32_t tl = (uint32_t)(32 * quarter) << 16;
+    const uint32_t tl = (uint32_t)(32 * q) << 16;
+    constexpr int HK = BN / 2;             // keys of a tile per thread
     auto wait_s = [&](uint64_t *b, uint32_t par) -> bool {
         return __all_sync(0xffffffffu, mbar_try_wait(b, par) || wait_bar(b, par, abort_flag, a.status));
     };
@@ -384,30 +433,34 @@ __device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter
         lv[p] = -CUDART_INF_F;
         li[p] = 0x7fffffff;
     }
-    float m_run = -CUDART_INF_F, l_run = 0.f;   // log2-domain running max and sum of this row
+    float m_run = -CUDART_INF_F, l_run = 0.f;   // log2-domain running max and sum of this half-row
     float m_acc = -CUDART_INF_F;                // max that o is expressed against
     float m_even = -CUDART_INF_F, m_odd = -CUDART_INF_F;   // the max P(j) was formed against, j even / odd
     float o[D];
 #pragma unroll
     for (int c = 0; c < D; ++c) o[c] = 0.f;
-    auto fold_o = [&](int i) -> bool {     // o += O(i), rescaled to the newer max
+    auto fold_o = [&](int i) -> bool {     // o += O_h(i), rescaled to the newer max
         if (!wait_s(&sh.o_full[i & 1], (i >> 1) & 1)) return false;
         fence_after();
-        float part[D];
-        tmem_ld32(tmem + 128 + 64 * (i & 1) + tl, part);
-        tmem_ld32(tmem + 128 + 64 * (i & 1) + 32 + tl, part + 32);
-        tmem_wait_ld();
+        const uint32_t to = tmem + 128 + 128 * (i & 1) + 64 * h + tl;
+        const float m_i = (i & 1) ? m_odd : m_even;
+        // (a half-row with no valid key yet has m = -inf and o = 0)
+        const float f = m_acc == -CUDART_INF_F ? 0.f : ex2(m_acc - m_i);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {   // 32 columns at a time (registers)
+            float part[32];
+            tmem_ld32(to + 32 * hh, part);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const float2 r2 = __ffma2_rn(make_float2(o[32 * hh + 2 * c], o[32 * hh + 2 * c + 1]), make_float2(f, f),
+                                             make_float2(part[2 * c], part[2 * c + 1]));
+                o[32 * hh + 2 * c] = r2.x;
+                o[32 * hh + 2 * c + 1] = r2.y;
+            }
+        }
         fence_before();
         mbar_arrive(&sh.o_free[i & 1]);
-        const float m_i = (i & 1) ? m_odd : m_even;
-        const float f = ex2(m_acc - m_i);
-#pragma unroll
-        for (int c = 0; c < D / 2; ++c) {
-            const float2 r2 = __ffma2_rn(make_float2(o[2 * c], o[2 * c + 1]), make_float2(f, f),
-                                         make_float2(part[2 * c], part[2 * c + 1]));
-            o[2 * c] = r2.x;
-            o[2 * c + 1] = r2.y;
-        }
         m_acc = m_i;
         return true;
     };
@@ -416,32 +469,33 @@ __device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter
         const int st = j & 1;
         if (!(ok = wait_s(&sh.s_full[st], (j >> 1) & 1))) break;
         fence_after();
-        float s[BN];                       // raw logits q̄·k̄ of keys j*64 .. j*64+63
-        tmem_ld32(tmem + 64 * st + tl, s);
-        tmem_ld32(tmem + 64 * st + 32 + tl, s + 32);
+        float s[HK];                       // raw logits q̄·k̄ of keys j*64 + 32h .. +31
+        tmem_ld32(tmem + 64 * st + 32 * h + tl, s);
         tmem_wait_ld();
         fence_before();
         mbar_arrive(&sh.s_free[st]);
-        const int key0 = j * BN;
-        if (key0 + BN > a.m) {
+        const int key0 = j * BN + HK * h;
+        if (key0 + HK > a.m) {
 #pragma unroll
-            for (int c = 0; c < BN; ++c)
+            for (int c = 0; c < HK; ++c)
                 if (key0 + c >= a.m) s[c] = -CUDART_INF_F;
         }
-        // ---- top-n: candidates beat the list's n-th entry; taken in key order.
-        //      The first tile seeds the list with its first NSEL logits, sorted.
+        // ---- top-n of this half's keys: candidates beat the list's n-th entry; taken in key
+        //      order. The first tile seeds the list with its first NSEL logits, sorted.
         int g0 = 0;
         if (j == 0) {
             sort_desc<NSEL>(s, lv, li);
+#pragma unroll
+            for (int p = 0; p < NSEL; ++p) li[p] += key0;
             g0 = NSEL / 8;
         }
-        float gm[BN / 8];                  // maxima of the 8 groups of 8 logits
+        float gm[HK / 8];                  // maxima of the 4 groups of 8 logits
 #pragma unroll
-        for (int g = 0; g < BN / 8; ++g)
+        for (int g = 0; g < HK / 8; ++g)
             gm[g] = fmax3(fmax3(s[8 * g], s[8 * g + 1], s[8 * g + 2]), fmax3(s[8 * g + 3], s[8 * g + 4], s[8 * g + 5]),
                           fmaxf(s[8 * g + 6], s[8 * g + 7]));
 #pragma unroll
-        for (int g = 0; g < BN / 8; ++g) {
+        for (int g = 0; g < HK / 8; ++g) {
             if (g < g0) continue;
             const float thr = lv[NSEL - 1];
             if (!(gm[g] > thr)) continue;  // no candidate in this group
@@ -459,64 +513,157 @@ __device__ void softmax_role(const Args &a, Smem &sh, uint32_t tmem, int quarter
                 if (v > lv[NSEL - 1]) list_insert<NSEL>(lv, li, v, key0 + 8 * g + u);
             }
         }
-        // ---- online softmax (log2 domain) of the row
-        const float mt = fmax3(fmax3(gm[0], gm[1], gm[2]), fmax3(gm[3], gm[4], gm[5]), fmaxf(gm[6], gm[7]));
+        // ---- online softmax (log2 domain) of the half-row
+        const float mt = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3]));
         const float m_new = fmaxf(m_run, mt * a.sl2);
+        const float m_sub = m_new == -CUDART_INF_F ? 0.f : m_new;   // no valid key yet: P = 0
         // exponents, then all exponentials, then four packed partial sums: in-order issue
         // never waits on one exp-unit result while later independent ones could be queued
         float ls;
         {
-            const float2 sc2 = make_float2(a.sl2, a.sl2), nm2 = make_float2(-m_new, -m_new);
+            const float2 sc2 = make_float2(a.sl2, a.sl2), nm2 = make_float2(-m_sub, -m_sub);
 #pragma unroll
-            for (int c = 0; c < BN / 2; ++c) {
+            for (int c = 0; c < HK / 2; ++c) {
                 const float2 x = __ffma2_rn(make_float2(s[2 * c], s[2 * c + 1]), sc2, nm2);
                 s[2 * c] = x.x;
                 s[2 * c + 1] = x.y;
             }
 #pragma unroll
-            for (int c = 0; c < BN; ++c) s[c] = ex2(s[c]);
+            for (int c = 0; c < HK; ++c) s[c] = ex2(s[c]);
             float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                               make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int c = 0; c < BN / 2; ++c) acc4[c & 3] = __fadd2_rn(acc4[c & 3], make_float2(s[2 * c], s[2 * c + 1]));
+            for (int c = 0; c < HK / 2; ++c) acc4[c & 3] = __fadd2_rn(acc4[c & 3], make_float2(s[2 * c], s[2 * c + 1]));
             const float2 t2 = __fadd2_rn(__fadd2_rn(acc4[0], acc4[1]), __fadd2_rn(acc4[2], acc4[3]));
             ls = t2.x + t2.y;
         }
-        l_run = fmaf(l_run, ex2(m_run - m_new), ls);
+        l_run = (m_run == -CUDART_INF_F ? 0.f : l_run * ex2(m_run - m_new)) + ls;
         m_run = m_new;
         if (st) m_odd = m_new;
         else m_even = m_new;
-        // ---- P(j) in tf32 parts, once P·V(j-1) has read the single P buffer
+        // ---- P(j) of this half in tf32 parts (region h of the P tile), once P·V(j-1) has read
+        //      the single P buffer
         if (!(ok = wait_s(&sh.p_empty, (j & 1) ^ 1))) break;
 #pragma unroll
-        for (int g = 0; g < 2; ++g)
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                store_split(sh.phi[g], sh.plo[g], sw128_offset(r, c),
-                            make_float4(s[32 * g + 4 * c], s[32 * g + 4 * c + 1], s[32 * g + 4 * c + 2],
-                                        s[32 * g + 4 * c + 3]));
+        for (int c = 0; c < 8; ++c)
+            store_split(sh.phi[h], sh.plo[h], sw128_offset(r, c),
+                        make_float4(s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]));
         fence_proxy_async();
         mbar_arrive(&sh.p_full);
         if (j > 0 && !(ok = fold_o(j - 1))) break;
     }
     if (ok && T > 0) ok = fold_o(T - 1);
-    if (row >= a.m) return;
-    int32_t *ix = a.idx + (int64_t)row * NSEL;
-    if (!ok) {                             // aborted: flag the rows for the selection kernel
+    // ---- half 1 hands (o, list, m, l) to half 0 through tensor memory: columns 384..447 (o),
+    //      448.. (list values), 480.. (list indices), 192 (m, l: half 1's own, now idle, O columns)
+    constexpr uint32_t kXO = 384, kXV = 448, kXI = 480, kXML = 192;
+    if (h == 1) {
+        if (ok) {
+            tmem_st32(tmem + kXO + tl, o);
+            tmem_st32(tmem + kXO + 32 + tl, o + 32);
 #pragma unroll
-        for (int p = 0; p < NSEL; ++p) ix[p] = -1;
+            for (int c = 0; c < NSEL; c += 16) {
+                float v16[16], i16[16];
+#pragma unroll
+                for (int p = 0; p < 16; ++p) {
+                    v16[p] = lv[c + p];
+                    i16[p] = __int_as_float(li[c + p]);
+                }
+                tmem_st16c(tmem + kXV + c + tl, v16);
+                tmem_st16c(tmem + kXI + c + tl, i16);
+            }
+            float ml[16];
+#pragma unroll
+            for (int p = 0; p < 16; ++p) ml[p] = p == 0 ? m_run : (p == 1 ? l_run : 0.f);
+            tmem_st16c(tmem + kXML + tl, ml);
+            tmem_wait_st();
+        }
+        fence_before();
+        mbar_arrive(&sh.merge[q]);         // (also when aborting: half 0 then sees the abort flag)
         return;
     }
-    const float inv = 1.f / l_run;
+    if (ok) ok = wait_s(&sh.merge[q], 0);
+    const bool live = row < a.m;           // rows past m are computed but not stored
+    int32_t *ix = a.idx + (int64_t)row * NSEL;
+    if (!ok) {                             // aborted: flag the rows for the selection kernel
+        if (live) {
+#pragma unroll
+            for (int p = 0; p < NSEL; ++p) ix[p] = -1;
+        }
+        return;
+    }
+    // the tensor-memory loads below are warp-collective (.sync.aligned): every lane of the warp
+    // takes part, rows past m included, and only the global stores are skipped for those
+    fence_after();
+    float mb, lb;
+    {
+        float ml[16];
+        tmem_ld16c(tmem + kXML + tl, ml);
+        tmem_wait_ld();
+        mb = ml[0];
+        lb = ml[1];
+    }
+    // ---- the two lists: keep, position by position, the better of this list's p-th and the
+    //      other's (NSEL-1-p)-th entry (a bitonic sequence holding the top NSEL of both), then sort
+#pragma unroll
+    for (int c = 0; c < NSEL; c += 16) {
+        float v16[16], i16[16];             // the other list's entries NSEL-1-c-15 .. NSEL-1-c
+        tmem_ld16c(tmem + kXV + (NSEL - 16 - c) + tl, v16);
+        tmem_ld16c(tmem + kXI + (NSEL - 16 - c) + tl, i16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int pp = 0; pp < 16; ++pp) {
+            const int p = c + pp;           // partner entry NSEL-1-p = (NSEL-16-c) + (15-pp)
+            const float w = v16[15 - pp];
+            const int k = __float_as_int(i16[15 - pp]);
+            if (ranks_before(w, k, lv[p], li[p])) {
+                lv[p] = w;
+                li[p] = k;
+            }
+        }
+    }
+    // bitonic merge of the NSEL entries into the selection order
+#pragma unroll
+    for (int jj = NSEL / 2; jj > 0; jj >>= 1)
+#pragma unroll
+        for (int p = 0; p < NSEL; ++p) {
+            const int pq = p ^ jj;
+            if (pq <= p) continue;
+            if (ranks_before(lv[pq], li[pq], lv[p], li[p])) {
+                const float tv = lv[p];
+                lv[p] = lv[pq];
+                lv[pq] = tv;
+                const int ti = li[p];
+                li[p] = li[pq];
+                li[pq] = ti;
+            }
+        }
+    if (live) {
+        int4 *idst = reinterpret_cast<int4 *>(ix);
+#pragma unroll
+        for (int p = 0; p < NSEL / 4; ++p) idst[p] = make_int4(li[4 * p], li[4 * p + 1], li[4 * p + 2], li[4 * p + 3]);
+    }
+    // ---- the softmax states: both halves rescaled to the larger maximum
+    const float m = fmaxf(m_run, mb);
+    const float fa = m_run == -CUDART_INF_F ? 0.f : ex2(m_run - m), fb = mb == -CUDART_INF_F ? 0.f : ex2(mb - m);
+    const float l = l_run * fa + lb * fb;
+    const float inv = 1.f / l;
     // training: natural-log log-sum-exp of the row's scaled logits
-    if (a.lse) a.lse[row] = (m_run + log2f(l_run)) * 0.69314718055994531f;
+    if (live && a.lse) a.lse[row] = (m + log2f(l)) * 0.69314718055994531f;
     float4 *dst = reinterpret_cast<float4 *>(a.o_cg + (int64_t)row * D);
 #pragma unroll
-    for (int c = 0; c < D / 4; ++c)
-        dst[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv, o[4 * c + 3] * inv);
-    int4 *idst = reinterpret_cast<int4 *>(ix);
+    for (int hh = 0; hh < 2; ++hh) {
+        float ob[32];
+        tmem_ld32(tmem + kXO + 32 * hh + tl, ob);
+        tmem_wait_ld();
+        if (!live) continue;
 #pragma unroll
-    for (int p = 0; p < NSEL / 4; ++p) idst[p] = make_int4(li[4 * p], li[4 * p + 1], li[4 * p + 2], li[4 * p + 3]);
+        for (int c = 0; c < 8; ++c) {
+            const int e = 32 * hh + 4 * c;
+            dst[8 * hh + c] = make_float4((o[e] * fa + ob[4 * c] * fb) * inv, (o[e + 1] * fa + ob[4 * c + 1] * fb) * inv,
+                                          (o[e + 2] * fa + ob[4 * c + 2] * fb) * inv,
+                                          (o[e + 3] * fa + ob[4 * c + 3] * fb) * inv);
+        }
+    }
 }
 
 template <int NSEL, bool PRE>
@@ -555,21 +702,22 @@ compress_tc_kernel(const float *__restrict__ qbar, const float *__restrict__ kba
         mbar_init(&sh.q_full, kFill);
         mbar_init(&sh.v_full, kFill);
         mbar_init(&sh.v_empty, 1);
-        mbar_init(&sh.p_full, 128);
+        mbar_init(&sh.p_full, 256);
         mbar_init(&sh.p_empty, 1);
         mbar_init(&sh.drain, 1);
         mbar_init(&sh.drain_pv, 1);
+        for (int qq = 0; qq < 4; ++qq) mbar_init(&sh.merge[qq], 32);
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sh.k_full[b], kFill);
             mbar_init(&sh.k_empty[b], 1);
             mbar_init(&sh.s_full[b], 1);
-            mbar_init(&sh.s_free[b], 128);
+            mbar_init(&sh.s_free[b], 256);
             mbar_init(&sh.o_full[b], 1);
-            mbar_init(&sh.o_free[b], 128);
+            mbar_init(&sh.o_free[b], 256);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 8) {
+    if (warp == 12) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&sh.tmem_base)),
                      "r"(TMEM_COLS)
@@ -581,26 +729,26 @@ compress_tc_kernel(const float *__restrict__ qbar, const float *__restrict__ kba
     fence_after();
     const uint32_t tmem = sh.tmem_base;
 
-    if (warp < 4) {
+    if (warp < 8) {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRowRegs));
-        softmax_role<NSEL>(a, sh, tmem, warp, lane, row0, T, abort_flag);
+        row_role<NSEL>(a, sh, tmem, warp & 3, warp >> 2, lane, row0, T, abort_flag);
     } else {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
         if (PRE) {
-            if (warp == 4 && lane == 0) copy_role(a, sh, row0, T, abort_flag);
-        } else if (warp < 8) {
-            convert_role(a, sh, threadIdx.x - 128, row0, T, abort_flag);
+            if (warp == 8 && lane == 0) copy_role(a, sh, row0, T, abort_flag);
+        } else if (warp < 12) {
+            convert_role(a, sh, threadIdx.x - 256, row0, T, abort_flag);
         }
-        if (warp == 8)
+        if (warp == 12)
             mma_s_role(a, sh, tmem, T, abort_flag);
-        else if (warp == 9)
+        else if (warp == 13)
             mma_pv_role(a, sh, tmem, T, abort_flag);
     }
     __syncwarp();
 
     fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == 12) {
         fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
                      : "memory");
