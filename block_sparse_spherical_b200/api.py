@@ -76,6 +76,64 @@ class BSA:
         return abi.bsa_check_status(self.workspace)
 
 
+class BSAStream:
+    """BSA forwards over a sequence of batches held in pinned host memory, with the host-device
+    copies overlapped with the computation.
+
+    run(batches, outs) enqueues, for batch i: its inputs copied in on a copy stream into device
+    buffer set i % 2, the forward (bsa_forward) on a compute stream, and its output copied back on
+    a third stream into outs[i]; so batch i+1's inputs move in and batch i-1's output moves out
+    while batch i computes. Events order the reuse of each buffer set (inputs: after the forward
+    two batches back has read them; output: after the copy-out two batches back has read it).
+    run returns once everything is enqueued; synchronize() waits for it.
+    """
+
+    def __init__(self, layer: BSA):
+        self.layer = layer
+        dev = layer.workspace.device
+        b, h, n, d = layer.shape
+        self.streams = [torch.cuda.Stream(dev) for _ in range(3)]   # copy in, compute, copy out
+        self.bufs = [dict(q=torch.empty(layer.shape, dtype=layer.dtype, device=dev),
+                          k=torch.empty(layer.shape, dtype=layer.dtype, device=dev),
+                          v=torch.empty(layer.shape, dtype=layer.dtype, device=dev),
+                          gates=torch.empty((b, h, n, 3), dtype=torch.float32, device=dev),
+                          out=torch.empty(layer.shape, dtype=layer.dtype, device=dev)) for _ in range(2)]
+        self.in_done = [torch.cuda.Event() for _ in range(2)]
+        self.cmp_done = [torch.cuda.Event() for _ in range(2)]
+        self.out_done = [torch.cuda.Event() for _ in range(2)]
+        self._used = [False, False]
+
+    def run(self, batches, outs) -> None:
+        s_in, s_cmp, s_out = self.streams
+        for i, ((q, k, v, gates), o) in enumerate(zip(batches, outs)):
+            for name, t in (("q", q), ("k", k), ("v", v), ("gates", gates), ("out", o)):
+                if t.is_cuda or not t.is_pinned():
+                    raise ValueError(f"{name} of batch {i} must be a pinned host tensor")
+            j = i % 2
+            buf = self.bufs[j]
+            with torch.cuda.stream(s_in):
+                if self._used[j]:
+                    s_in.wait_event(self.cmp_done[j])
+                for name, t in (("q", q), ("k", k), ("v", v), ("gates", gates)):
+                    buf[name].copy_(t, non_blocking=True)
+                self.in_done[j].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(self.in_done[j])
+                if self._used[j]:
+                    s_cmp.wait_event(self.out_done[j])
+                self.layer(buf["q"], buf["k"], buf["v"], buf["gates"], out=buf["out"])
+                self.cmp_done[j].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(self.cmp_done[j])
+                o.copy_(buf["out"], non_blocking=True)
+                self.out_done[j].record(s_out)
+            self._used[j] = True
+
+    def synchronize(self) -> None:
+        for st in self.streams:
+            st.synchronize()
+
+
 class BSATrain(BSA):
     """A BSA layer of fixed shape for training: forward() saves what backward() needs.
 

@@ -256,3 +256,26 @@ def test_mirrored_output_stores():
     assert abi.bsa_check_status(ws) == 0
     for t in [out] + mirrors:
         assert torch.equal(t, want)
+
+
+def test_stream_matches_forward():
+    """api.BSAStream (host copies overlapped with the computation, two device buffer sets) gives,
+    for every batch of a sequence, exactly the output of api.BSA on that batch."""
+    cfg = CONFIGS["nside32"]
+    q, k, v, g = parity.device_inputs(cfg)
+    bsa = api.BSA.from_config(cfg)
+    batches, want = [], []
+    for i in range(5):
+        f = 1.0 + 0.25 * i                          # distinct batches: q scaled (exact in bf16)
+        qi = (q.float() * f).to(torch.bfloat16)
+        gi = torch.roll(g, shifts=i, dims=2).contiguous()
+        want.append(bsa(qi, k, v, gi).cpu())
+        batches.append(tuple(t.cpu().pin_memory() for t in (qi, k, v, gi)))
+    torch.cuda.synchronize()
+    outs = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(5)]
+    pipe = api.BSAStream(bsa)
+    pipe.run(batches, outs)
+    pipe.synchronize()
+    assert bsa.check_status() == 0
+    for i in range(5):
+        assert torch.equal(outs[i], want[i]), f"batch {i} differs"
