@@ -86,6 +86,50 @@ template <> __device__ __forceinline__ float load1<__nv_bfloat16>(const __nv_bfl
     return __bfloat162float(*p);
 }
 
+// N consecutive elements (N = 2, 4 or 8; at an offset that is a multiple of N) as floats, with one
+// 4-, 8- or 16-byte load for bf16 (two for 8 fp32), and the same for stores.
+template <int N> struct VecU32;
+template <> struct VecU32<1> { using type = uint32_t; };
+template <> struct VecU32<2> { using type = uint2; };
+template <> struct VecU32<4> { using type = uint4; };
+template <int N>
+__device__ __forceinline__ void loadv(const __nv_bfloat16 *p, float *f) {
+    using V = typename VecU32<N / 2>::type;
+    const V w = __ldg(reinterpret_cast<const V *>(p));
+    const uint32_t *u = reinterpret_cast<const uint32_t *>(&w);
+#pragma unroll
+    for (int e = 0; e < N / 2; ++e) {
+        f[2 * e] = __uint_as_float(u[e] << 16);
+        f[2 * e + 1] = __uint_as_float(u[e] & 0xffff0000u);
+    }
+}
+template <int N>
+__device__ __forceinline__ void loadv(const float *p, float *f) {
+#pragma unroll
+    for (int e = 0; e < N; e += 2) {
+        const float2 w = __ldg(reinterpret_cast<const float2 *>(p + e));
+        f[e] = w.x;
+        f[e + 1] = w.y;
+    }
+}
+template <int N>
+__device__ __forceinline__ void storev(__nv_bfloat16 *p, const float *f) {
+    using V = typename VecU32<N / 2>::type;
+    V w;
+    uint32_t *u = reinterpret_cast<uint32_t *>(&w);
+#pragma unroll
+    for (int e = 0; e < N / 2; ++e) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(f[2 * e], f[2 * e + 1]);
+        u[e] = *reinterpret_cast<const uint32_t *>(&b2);
+    }
+    *reinterpret_cast<V *>(p) = w;
+}
+template <int N>
+__device__ __forceinline__ void storev(float *p, const float *f) {
+#pragma unroll
+    for (int e = 0; e < N; e += 2) *reinterpret_cast<float2 *>(p + e) = make_float2(f[e], f[e + 1]);
+}
+
 // kappa[b][j][e] = s·log2(e) · Σ_c W_q[c][e] k[b][j][c]: each source key seen from position
 // space, so that the logit of (i, j) is p_ij · kappa_j (= s (W_q p_ij)·k_j). One warp per source
 // point, lane l holding channels l*C .. l*C+C-1.
@@ -162,13 +206,12 @@ interp_kernel(int64_t batch, int64_t n_tgt, int64_t n_src, const int32_t *__rest
             for (int jj = 0; jj < KN; ++jj) {
                 const float pw = __shfl_sync(half, pj, (lane & 16) | jj);
                 const int32_t sj = __shfl_sync(half, src, (lane & 16) | jj);
-                const T *vr = vb + (int64_t)sj * D + j * C4;
+                float vv[C4];
+                loadv<C4>(vb + (int64_t)sj * D + j * C4, vv);   // one vector load per neighbour
 #pragma unroll
-                for (int c = 0; c < C4; ++c) acc[c] = fmaf(pw, load1<T>(vr + c), acc[c]);
+                for (int c = 0; c < C4; ++c) acc[c] = fmaf(pw, vv[c], acc[c]);
             }
-            T *o = out + (b * n_tgt + i) * D + j * C4;
-#pragma unroll
-            for (int c = 0; c < C4; ++c) o[c] = from_f32<T>(acc[c]);
+            storev<C4>(out + (b * n_tgt + i) * D + j * C4, acc);
         }
     }
 }
