@@ -80,12 +80,6 @@ healpix_plan_kernel(int64_t nside, int64_t nlat, int64_t nlon, int32_t *__restri
     }
 }
 
-template <typename T> __device__ __forceinline__ float load1(const T *p);
-template <> __device__ __forceinline__ float load1<float>(const float *p) { return __ldg(p); }
-template <> __device__ __forceinline__ float load1<__nv_bfloat16>(const __nv_bfloat16 *p) {
-    return __bfloat162float(*p);
-}
-
 // N consecutive elements (N = 2, 4 or 8; at an offset that is a multiple of N) as floats, with one
 // 4-, 8- or 16-byte load for bf16 (two for 8 fp32), and the same for stores.
 template <int N> struct VecU32;
@@ -131,40 +125,34 @@ __device__ __forceinline__ void storev(float *p, const float *f) {
 }
 
 // kappa[b][j][e] = s·log2(e) · Σ_c W_q[c][e] k[b][j][c]: each source key seen from position
-// space, so that the logit of (i, j) is p_ij · kappa_j (= s (W_q p_ij)·k_j). One warp per source
-// point, lane l holding channels l*C .. l*C+C-1.
+// space, so that the logit of (i, j) is p_ij · kappa_j (= s (W_q p_ij)·k_j). One thread per
+// source point (its row read with 16-byte vector loads, W_q from shared memory): an HBM stream.
 template <typename T, int C>
 __global__ void __launch_bounds__(256)
 kappa_kernel(int64_t rows, const float *__restrict__ wq, const T *__restrict__ ksrc, float *__restrict__ kappa,
              float scale_log2) {
     constexpr int D = 32 * C;
-    const int lane = threadIdx.x & 31;
-    float w[C][3];
-#pragma unroll
-    for (int c = 0; c < C; ++c)
-#pragma unroll
-        for (int e = 0; e < 3; ++e) w[c][e] = __ldg(wq + (lane * C + c) * 3 + e);
-    for (int64_t r = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; r < rows;
-         r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    __shared__ float w[D * 3];
+    for (int e = threadIdx.x; e < D * 3; e += blockDim.x) w[e] = __ldg(wq + e);
+    __syncthreads();
+    for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows; r += (int64_t)gridDim.x * blockDim.x) {
+        const T *kr = ksrc + r * D;
         float a0 = 0.f, a1 = 0.f, a2 = 0.f;
 #pragma unroll
-        for (int c = 0; c < C; ++c) {
-            const float kc = load1<T>(ksrc + r * D + lane * C + c);
-            a0 = fmaf(w[c][0], kc, a0);
-            a1 = fmaf(w[c][1], kc, a1);
-            a2 = fmaf(w[c][2], kc, a2);
-        }
+        for (int c0 = 0; c0 < D; c0 += 8) {
+            float kv[8];
+            loadv<8>(kr + c0, kv);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            a0 += __shfl_xor_sync(0xffffffffu, a0, off);
-            a1 += __shfl_xor_sync(0xffffffffu, a1, off);
-            a2 += __shfl_xor_sync(0xffffffffu, a2, off);
+            for (int e = 0; e < 8; ++e) {
+                const float *wc = w + (c0 + e) * 3;
+                a0 = fmaf(wc[0], kv[e], a0);
+                a1 = fmaf(wc[1], kv[e], a1);
+                a2 = fmaf(wc[2], kv[e], a2);
+            }
         }
-        if (lane == 0) {
-            kappa[r * 3] = a0 * scale_log2;
-            kappa[r * 3 + 1] = a1 * scale_log2;
-            kappa[r * 3 + 2] = a2 * scale_log2;
-        }
+        kappa[r * 3] = a0 * scale_log2;
+        kappa[r * 3 + 1] = a1 * scale_log2;
+        kappa[r * 3 + 2] = a2 * scale_log2;
     }
 }
 
@@ -224,8 +212,9 @@ cudaError_t launch_interp_t(int64_t batch, int64_t n_tgt, int64_t n_src, int64_t
     const T *kt = static_cast<const T *>(k), *vt = static_cast<const T *>(v);
     T *ot = static_cast<T *>(out);
     const int64_t krows = batch * n_src;
-    int64_t kctas = (krows * 32 + 255) / 256;
+    int64_t kctas = (krows + 255) / 256;
     if (kctas > 148 * 32) kctas = 148 * 32;
+    if (kctas < 1) kctas = 1;
     int64_t ctas = (n_tgt * 16 + 255) / 256;
     if (ctas > 148 * 64) ctas = 148 * 64;
     if (ctas < 1) ctas = 1;
