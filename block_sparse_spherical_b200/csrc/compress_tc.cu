@@ -11,8 +11,9 @@
 // into one fp32 accumulator in TMEM. The dropped a_lo·b_lo term and the
 // truncated low bits of the remainders leave a relative error below 2^-19 per
 // product, so the logits that decide the ranking stay far inside its 1e-4
-// margin. Each tile's P·V is a fresh accumulation of 24 MMAs; the tiles are
-// summed in fp32 registers.
+// margin. Each tile's P·V is a fresh accumulation (12 MMAs for each half of
+// its keys, into the half's own TMEM columns); the tiles are summed in fp32
+// registers.
 //
 // One CTA owns 128 query blocks (rows) of one slab and streams the slab's key
 // blocks in tiles of 64 (the m×m logit matrix never leaves the SM):
