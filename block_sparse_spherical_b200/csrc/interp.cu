@@ -175,9 +175,17 @@ interp_kernel(int64_t batch, int64_t n_tgt, int64_t n_src, const int32_t *__rest
         const float *pr = rel + (i * KN + j) * 3;
         const float p0 = __ldg(pr), p1 = __ldg(pr + 1), p2 = __ldg(pr + 2);
         if (__any_sync(half, bad) && j == 0 && status) atomicOr(status, kStatusBadIndex);
+        // kappa of the next batch image is loaded while this one's rows are gathered
+        const float *kp0 = kappa + src * 3;
+        float k0 = __ldg(kp0), k1 = __ldg(kp0 + 1), k2 = __ldg(kp0 + 2);
         for (int64_t b = 0; b < batch; ++b) {
-            const float *kp = kappa + (b * n_src + src) * 3;
-            float lg = fmaf(p0, __ldg(kp), fmaf(p1, __ldg(kp + 1), p2 * __ldg(kp + 2)));
+            float lg = fmaf(p0, k0, fmaf(p1, k1, p2 * k2));
+            if (b + 1 < batch) {
+                const float *kp = kappa + ((b + 1) * n_src + src) * 3;
+                k0 = __ldg(kp);
+                k1 = __ldg(kp + 1);
+                k2 = __ldg(kp + 2);
+            }
             float mx = lg;
 #pragma unroll
             for (int off = 8; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(half, mx, off));
