@@ -408,6 +408,7 @@ def ring_scheme_centres(nside):
 
 def unit(zphi):
     z, ph = zphi[:, 0], zphi[:, 1]
+    assert np.all(np.isfinite(zphi)) and np.all(np.abs(z) <= 1), "a point off the sphere (|z| > 1 or not finite)"
     st = np.sqrt(1 - z * z)
     return np.stack([st * np.cos(ph), st * np.sin(ph), z], 1)
 
