@@ -47,7 +47,7 @@ def test_plan_matches_oracle(nside, nlat, nlon):
 
 @pytest.mark.parametrize("nside,nlat,nlon,d,dtype,batch", [
     (32, 121, 240, 64, torch.float32, 2),     # 1.5 degree source onto Nside 32
-    (32, 121, 240, 64, torch.bfloat16, 2),
+    (32, 121, 240, 64, torch.bfloat16, 3),    # odd batch: the next image's kappa is loaded ahead
     (16, 61, 120, 32, torch.float32, 1),
     (16, 61, 120, 128, torch.bfloat16, 1),
     (256, 721, 1440, 64, torch.bfloat16, 1),  # 0.25 degree source onto Nside 256 (786,432 pixels)
