@@ -85,7 +85,10 @@ class BSAStream:
     a third stream into outs[i]; so batch i+1's inputs move in and batch i-1's output moves out
     while batch i computes. Events order the reuse of each buffer set (inputs: after the forward
     two batches back has read them; output: after the copy-out two batches back has read it).
-    run returns once everything is enqueued; synchronize() waits for it.
+    run returns once everything is enqueued; synchronize() waits for it. The host tensors must
+    stay alive and unchanged until then. The device buffers (and the layer's workspace and index
+    array) are marked as used by the streams that touch them, so that memory freed with this object
+    is not handed out again while a copy or a forward on one of them is still pending.
     """
 
     def __init__(self, layer: BSA):
@@ -98,6 +101,12 @@ class BSAStream:
                           v=torch.empty(layer.shape, dtype=layer.dtype, device=dev),
                           gates=torch.empty((b, h, n, 3), dtype=torch.float32, device=dev),
                           out=torch.empty(layer.shape, dtype=layer.dtype, device=dev)) for _ in range(2)]
+        for buf in self.bufs:
+            for t in buf.values():
+                for st in self.streams:
+                    t.record_stream(st)
+        layer.workspace.record_stream(self.streams[1])
+        layer.sel_idx.record_stream(self.streams[1])
         self.in_done = [torch.cuda.Event() for _ in range(2)]
         self.cmp_done = [torch.cuda.Event() for _ in range(2)]
         self.out_done = [torch.cuda.Event() for _ in range(2)]
