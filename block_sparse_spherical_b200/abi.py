@@ -88,10 +88,14 @@ def make_config(cfg, scale: float = 0.0) -> BsaConfig:
 
 
 def _ptr(t) -> int | None:
+    """Address of a device buffer: None, a raw address, or a CUDA tensor (a host tensor is refused:
+    every buffer argument of the library is device memory)."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_cuda:
+        raise ValueError("buffer arguments must be CUDA tensors (device memory), got a host tensor")
     return t.data_ptr()
 
 

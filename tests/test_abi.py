@@ -132,3 +132,15 @@ def test_python_binding_raises_on_error(lib):
     with pytest.raises(abi.BsaError) as e:
         abi.bsa_workspace_size(c)
     assert e.value.code == 1
+
+
+def test_python_binding_refuses_host_tensors(lib):
+    """Every buffer of the library is device memory: the binding refuses a host tensor before the
+    library is called (no host pointer ever reaches a kernel)."""
+    import torch
+    c = cfg_of()
+    t = torch.zeros(16, dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        abi.bsa_pool(c, t, t, t, t, t, t, stream=0)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        abi.bsa_check_status(t)
